@@ -1,0 +1,234 @@
+// C ABI of libnabla.so (declared in include/nabla.h): argument checks,
+// workspace layout, status word, kernel dispatch.  Every host-detectable
+// error is returned before anything is enqueued.
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/nabla.h"
+#include "common.cuh"
+
+// launchers (mask.cu, flatten.cu, attn_*.cu)
+cudaError_t nabla_launch_flatten(const void *in, void *out, int64_t outer, int T, int H, int W,
+                                 int P, int64_t inner_bytes, int inverse, cudaStream_t stream);
+cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, float p,
+                                    float scale, int wt, int wh, int ww, unsigned flags,
+                                    const void *q, const void *k, float *qbar, float *kbar_t,
+                                    uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
+                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream);
+cudaError_t nabla_launch_attn_fwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
+                                      const void *k, const void *v, const uint16_t *row_idx,
+                                      const int32_t *row_cnt, void *o, float *lse,
+                                      cudaStream_t stream);
+cudaError_t nabla_launch_attn_bwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
+                                      const void *k, const void *v, const void *o,
+                                      const void *dout, const float *lse, const uint16_t *row_idx,
+                                      const int32_t *row_cnt, const uint16_t *col_idx,
+                                      const int32_t *col_cnt, void *dq, void *dk, void *dv,
+                                      float *dl, cudaStream_t stream);
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr int kMaxNb = 2048;
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Dims {
+    int64_t BH, N;
+    int nb, D, Hp, Wp;
+};
+
+int check_shape(const nabla_shape *s, Dims *d) {
+    if (s == nullptr) return NABLA_ERR_NULL;
+    if (s->B < 1 || s->heads < 1 || s->T < 1 || s->H < 1 || s->W < 1) return NABLA_ERR_SHAPE;
+    if (s->P != 8 || s->H % s->P != 0 || s->W % s->P != 0) return NABLA_ERR_SHAPE;
+    if (s->D != 64 && s->D != 128) return NABLA_ERR_SHAPE;
+    const int64_t nb = static_cast<int64_t>(s->T) * (s->H / s->P) * (s->W / s->P);
+    if (nb < 1 || nb > kMaxNb) return NABLA_ERR_SHAPE;
+    d->BH = static_cast<int64_t>(s->B) * s->heads;
+    d->nb = static_cast<int>(nb);
+    d->N = nb * nabla::kBlk;
+    d->D = s->D;
+    d->Hp = s->H / s->P;
+    d->Wp = s->W / s->P;
+    return NABLA_OK;
+}
+
+int check_params(const nabla_params *p, bool need_window) {
+    if (p == nullptr) return NABLA_ERR_NULL;
+    if (!(p->p >= 0.f && p->p <= 1.f)) return NABLA_ERR_PARAM;  // also rejects NaN
+    if (!(p->scale > 0.f) || !std::isfinite(p->scale)) return NABLA_ERR_PARAM;
+    if ((p->flags & ~(NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS)) != 0) return NABLA_ERR_PARAM;
+    if ((p->flags & NABLA_NO_STA) && (p->flags & NABLA_FULL_STA)) return NABLA_ERR_PARAM;
+    if (need_window && !(p->flags & (NABLA_NO_STA | NABLA_FULL_STA))) {
+        for (int w : {p->sta_t, p->sta_h, p->sta_w})
+            if (w < 1 || (w & 1) == 0) return NABLA_ERR_PARAM;
+    }
+    return NABLA_OK;
+}
+
+size_t ws_bytes(const Dims &d, int op) {
+    switch (op) {
+        case NABLA_OP_BUILD_MASK:
+            return kStatusBytes + 2 * round256(sizeof(float) * d.BH * d.nb * d.D);
+        case NABLA_OP_ATTN_FWD:
+            return kStatusBytes;
+        case NABLA_OP_ATTN_BWD:
+            return kStatusBytes + round256(sizeof(float) * d.BH * d.N);
+        default:
+            return 0;
+    }
+}
+
+int check_ws(const Dims &d, int op, void *ws, size_t bytes) {
+    if (ws == nullptr || bytes < ws_bytes(d, op)) return NABLA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return NABLA_ERR_ALIGN;
+    return NABLA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? NABLA_OK : NABLA_ERR_CUDA; }
+
+int clear_status(void *ws, cudaStream_t s) {
+    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(int), s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int nabla_flatten(const void *in, void *out, int64_t outer, int T, int H, int W, int P,
+                  int64_t inner_bytes, int inverse, nabla_stream_t stream) {
+    if (outer < 0 || T < 0 || H < 0 || W < 0 || P < 1 || inner_bytes < 0) return NABLA_ERR_SHAPE;
+    if (H % P != 0 || W % P != 0) return NABLA_ERR_SHAPE;
+    if (inner_bytes % 16 != 0) return NABLA_ERR_ALIGN;
+    if (outer == 0 || T == 0 || H == 0 || W == 0 || inner_bytes == 0) return NABLA_OK;  // empty
+    if (in == nullptr || out == nullptr) return NABLA_ERR_NULL;
+    if (!aligned16(in) || !aligned16(out)) return NABLA_ERR_ALIGN;
+    if (in == out) return NABLA_ERR_PARAM;
+    return cuda_status(nabla_launch_flatten(in, out, outer, T, H, W, P, inner_bytes, inverse,
+                                            reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t nabla_workspace_size(const nabla_shape *shape, int op) {
+    Dims d;
+    if (check_shape(shape, &d) != NABLA_OK) return 0;
+    return ws_bytes(d, op);
+}
+
+size_t nabla_mask_bytes(const nabla_shape *shape, int part) {
+    Dims d;
+    if (check_shape(shape, &d) != NABLA_OK) return 0;
+    const size_t rows = static_cast<size_t>(d.BH) * d.nb;
+    switch (part) {
+        case NABLA_MASK_BITS:
+            return rows * ((d.nb + 31) / 32) * sizeof(uint32_t);
+        case NABLA_MASK_ROW_IDX:
+        case NABLA_MASK_COL_IDX:
+            return rows * d.nb * sizeof(uint16_t);
+        case NABLA_MASK_ROW_CNT:
+        case NABLA_MASK_COL_CNT:
+            return rows * sizeof(int32_t);
+        default:
+            return 0;
+    }
+}
+
+int nabla_build_mask(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
+                     const nabla_bf16 *k, const nabla_mask *mask, void *workspace,
+                     size_t workspace_bytes, nabla_stream_t stream) {
+    Dims d;
+    int st = check_shape(shape, &d);
+    if (st != NABLA_OK) return st;
+    if ((st = check_params(params, true)) != NABLA_OK) return st;
+    if (q == nullptr || k == nullptr || mask == nullptr || mask->bits == nullptr ||
+        mask->row_idx == nullptr || mask->row_cnt == nullptr)
+        return NABLA_ERR_NULL;
+    const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
+    if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k)) return NABLA_ERR_ALIGN;
+    if ((st = check_ws(d, NABLA_OP_BUILD_MASK, workspace, workspace_bytes)) != NABLA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
+    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
+    float *qbar = reinterpret_cast<float *>(w);
+    float *kbar_t = reinterpret_cast<float *>(w + round256(sizeof(float) * d.BH * d.nb * d.D));
+    return cuda_status(nabla_launch_build_mask(
+        d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
+        params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
+        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr, s));
+}
+
+int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
+                   const nabla_bf16 *k, const nabla_bf16 *v, const nabla_mask *mask,
+                   nabla_bf16 *o, float *lse, void *workspace, size_t workspace_bytes,
+                   nabla_stream_t stream) {
+    Dims d;
+    int st = check_shape(shape, &d);
+    if (st != NABLA_OK) return st;
+    if ((st = check_params(params, false)) != NABLA_OK) return st;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || mask == nullptr ||
+        mask->row_idx == nullptr || mask->row_cnt == nullptr)
+        return NABLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return NABLA_ERR_ALIGN;
+    if ((st = check_ws(d, NABLA_OP_ATTN_FWD, workspace, workspace_bytes)) != NABLA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
+    return cuda_status(nabla_launch_attn_fwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v,
+                                                 mask->row_idx, mask->row_cnt, o, lse, s));
+}
+
+int nabla_attn_bwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
+                   const nabla_bf16 *k, const nabla_bf16 *v, const nabla_bf16 *o,
+                   const nabla_bf16 *dout, const float *lse, const nabla_mask *mask,
+                   nabla_bf16 *dq, nabla_bf16 *dk, nabla_bf16 *dv, void *workspace,
+                   size_t workspace_bytes, nabla_stream_t stream) {
+    Dims d;
+    int st = check_shape(shape, &d);
+    if (st != NABLA_OK) return st;
+    if ((st = check_params(params, false)) != NABLA_OK) return st;
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || dout == nullptr ||
+        lse == nullptr || dq == nullptr || dk == nullptr || dv == nullptr || mask == nullptr ||
+        mask->row_idx == nullptr || mask->row_cnt == nullptr || mask->col_idx == nullptr ||
+        mask->col_cnt == nullptr)
+        return NABLA_ERR_NULL;
+    for (const void *p : {static_cast<const void *>(q), static_cast<const void *>(k),
+                          static_cast<const void *>(v), static_cast<const void *>(o),
+                          static_cast<const void *>(dout), static_cast<const void *>(dq),
+                          static_cast<const void *>(dk), static_cast<const void *>(dv)})
+        if (!aligned16(p)) return NABLA_ERR_ALIGN;
+    if ((st = check_ws(d, NABLA_OP_ATTN_BWD, workspace, workspace_bytes)) != NABLA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
+    float *dl = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + kStatusBytes);
+    return cuda_status(nabla_launch_attn_bwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v, o,
+                                                 dout, lse, mask->row_idx, mask->row_cnt,
+                                                 mask->col_idx, mask->col_cnt, dq, dk, dv, dl, s));
+}
+
+int nabla_status(const void *workspace, nabla_stream_t stream) {
+    if (workspace == nullptr) return NABLA_ERR_NULL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return NABLA_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NABLA_ERR_CUDA;
+    return word == nabla::kDevOk ? NABLA_OK : NABLA_ERR_TIMEOUT;
+}
+
+const char *nabla_strerror(int status) {
+    switch (status) {
+        case NABLA_OK: return "ok";
+        case NABLA_ERR_SHAPE: return "unsupported or inconsistent shape";
+        case NABLA_ERR_ALIGN: return "pointer or byte count not 16-byte aligned";
+        case NABLA_ERR_PARAM: return "invalid parameter";
+        case NABLA_ERR_WORKSPACE: return "workspace missing or too small";
+        case NABLA_ERR_CUDA: return "CUDA call or kernel launch failed";
+        case NABLA_ERR_TIMEOUT: return "device-side bounded wait expired";
+        case NABLA_ERR_NULL: return "required pointer is NULL";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,411 @@
+// Adaptive block mask ("NABLA: Neighborhood Adaptive Block-Level Attention",
+// section 手法: NABLA, "適応型マスク構築 (ブロックレベル・プーリング & CDF 閾値処理)"
+// and "STA とのハイブリッド統合").
+//
+//   pool_kernel        block means of Q and K (64 tokens -> one fp32 row),
+//                      float32 running sum in ascending token order, * 1/64.
+//                      Q-bar row-major [BH, nb, D]; K-bar transposed
+//                      [BH, D, nb] so the score kernel streams it coalesced.
+//   score_cut_kernel   per (bh, 16 query blocks): pooled scores as a float32
+//                      fma chain over d ascending (register-tiled FFMA; the
+//                      order per output is the plain ascending chain), then
+//                      per row: weights exp(s - max) in float64, integer mass
+//                      floor(w * 2^40), a radix select over the 48-bit key
+//                      (score bits, then inverted block index) that finds the
+//                      last block of the shortest descending prefix whose mass
+//                      reaches p * total, and the OR with the STA window and
+//                      the diagonal.  Writes the bit row and the ascending row
+//                      list.
+//   col_lists_kernel   transpose of the bit rows into ascending column lists.
+//
+// The mass sums are exact integers, so the selected set does not depend on
+// the order in which threads add them.
+#include "common.cuh"
+
+namespace nabla {
+
+// ---------------------------------------------------------------------------
+// pooling
+// ---------------------------------------------------------------------------
+// CTA = 256 threads = (256 / CH) blocks x CH chunks of 8 features, CH = D/8.
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                   const __nv_bfloat16 *__restrict__ k,
+                                                   float *__restrict__ qbar,
+                                                   float *__restrict__ kbar_t, int64_t BH,
+                                                   int nb) {
+    constexpr int CH = D / 8;
+    constexpr int BPC = 256 / CH;  // blocks per CTA
+    __shared__ float tile[BPC][D + 1];
+    const int tid = threadIdx.x;
+    const int c = tid % CH;
+    const int bl = tid / CH;
+    const int tiles_per_head = (nb + BPC - 1) / BPC;
+    const int64_t cta = blockIdx.x;
+    const int which = static_cast<int>(cta / (BH * tiles_per_head));  // 0: q, 1: k
+    const int64_t rem = cta % (BH * tiles_per_head);
+    const int64_t bh = rem / tiles_per_head;
+    const int i0 = static_cast<int>(rem % tiles_per_head) * BPC;
+    const int i = i0 + bl;
+    const __nv_bfloat16 *x = which ? k : q;
+    const int64_t N = static_cast<int64_t>(nb) * kBlk;
+
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    if (i < nb) {
+        const int4 *src =
+            reinterpret_cast<const int4 *>(x + (bh * N + static_cast<int64_t>(i) * kBlk) * D) + c;
+#pragma unroll 1
+        for (int r0 = 0; r0 < kBlk; r0 += 16) {
+            int4 v[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) v[r] = __ldg(src + (r0 + r) * CH);
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v[r]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 f = __bfloat1622float2(h[e]);
+                    acc[2 * e] = __fadd_rn(acc[2 * e], f.x);
+                    acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], f.y);
+                }
+            }
+        }
+    }
+    const float inv = 1.0f / kBlk;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = __fmul_rn(acc[e], inv);
+    if (which == 0) {
+        if (i < nb) {
+            float4 *dst = reinterpret_cast<float4 *>(qbar + (bh * nb + i) * D + c * 8);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tile[bl][c * 8 + e] = acc[e];
+        __syncthreads();
+        // write [D][nb]: each thread writes consecutive blocks of one feature
+        for (int idx = tid; idx < D * BPC; idx += 256) {
+            const int d = idx / BPC, b = idx % BPC;
+            if (i0 + b < nb) kbar_t[(bh * D + d) * nb + i0 + b] = tile[b][d];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// scores + CDF cut + STA + lists
+// ---------------------------------------------------------------------------
+constexpr int kRows = 16;    // query blocks per CTA
+constexpr int kCols = 256;   // key blocks per score tile
+constexpr int kDc = 32;      // features per staged K-bar slice
+constexpr int kThreads = 256;
+
+struct CutParams {
+    int nb, Hp, Wp, wt, wh, ww;
+    unsigned flags;
+    float p, scale;
+};
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+    uint32_t b = __float_as_uint(s);
+    if (b == 0x80000000u) b = 0u;  // -0 ranks with +0
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ uint64_t mass_of(float s, float smax) {
+    const double w = exp(static_cast<double>(s) - static_cast<double>(smax));
+    return __double2ull_rz(w * 1099511627776.0);  // * 2^40, exact scaling
+}
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+    uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v), src);
+    uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), src);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_up_u64(uint64_t v, int d) {
+    uint32_t lo = __shfl_up_sync(0xffffffffu, static_cast<uint32_t>(v), d);
+    uint32_t hi = __shfl_up_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), d);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    score_cut_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar_t,
+                     CutParams prm, uint32_t *__restrict__ bits, uint16_t *__restrict__ row_idx,
+                     int32_t *__restrict__ row_cnt) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int nb = prm.nb;
+    const int nbp = (nb + 3) & ~3;
+    float *sS = reinterpret_cast<float *>(smem);                       // [kRows][nbp]
+    unsigned char *work = smem + sizeof(float) * kRows * nbp;          // phase-specific
+    float *sQt = reinterpret_cast<float *>(work);                      // [D][kRows]
+    float *sKt = sQt + D * kRows;                                      // [kDc][kCols]
+    uint64_t *hmass = reinterpret_cast<uint64_t *>(work);              // [8 warps][256]
+    uint32_t *hcnt = reinterpret_cast<uint32_t *>(hmass + 8 * 256);    // [8 warps][256]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tiles = (nb + kRows - 1) / kRows;
+    const int64_t bh = blockIdx.x / tiles;
+    const int i0 = (blockIdx.x % tiles) * kRows;
+
+    // ---- phase 1: scores s[r][j] = (fma chain over d of qbar_i . kbar_j) * scale
+    for (int idx = tid; idx < kRows * D; idx += kThreads) {
+        const int r = idx / D, d = idx % D;
+        sQt[d * kRows + r] = (i0 + r < nb) ? qbar[(bh * nb + i0 + r) * D + d] : 0.f;
+    }
+    const int cg = tid % 64;  // 4 consecutive columns
+    const int rg = tid / 64;  // 4 consecutive rows
+    const float *kt = kbar_t + bh * static_cast<int64_t>(D) * nb;
+    for (int j0 = 0; j0 < nb; j0 += kCols) {
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        for (int d0 = 0; d0 < D; d0 += kDc) {
+            __syncthreads();
+            for (int idx = tid; idx < kDc * kCols; idx += kThreads) {
+                const int d = idx / kCols, j = idx % kCols;
+                sKt[idx] = (j0 + j < nb) ? kt[static_cast<int64_t>(d0 + d) * nb + j0 + j] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 8
+            for (int d = 0; d < kDc; ++d) {
+                const float4 qv = *reinterpret_cast<const float4 *>(sQt + (d0 + d) * kRows + rg * 4);
+                const float4 kv = *reinterpret_cast<const float4 *>(sKt + d * kCols + cg * 4);
+                const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+                const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(qa[a], ka[b], acc[a][b]);
+            }
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int j = j0 + cg * 4 + b;
+                if (j < nb) sS[(rg * 4 + a) * nbp + j] = __fmul_rn(acc[a][b], prm.scale);
+            }
+    }
+    __syncthreads();
+
+    // ---- phase 2: one warp per row
+    uint64_t *hm = hmass + warp * 256;
+    uint32_t *hc = hcnt + warp * 256;
+    const int words = (nb + 31) >> 5;
+    const bool keep_all = prm.p >= 1.0f;
+    const bool keep_none = prm.p <= 0.0f;
+    for (int r = warp; r < kRows; r += kThreads / 32) {
+        const int i = i0 + r;
+        if (i >= nb) break;
+        const float *srow = sS + r * nbp;
+        uint64_t cstar = 0;  // composite key of the last kept block
+        if (!keep_all && !keep_none) {
+            float smax = -INFINITY;
+            for (int j = lane; j < nb; j += 32) smax = fmaxf(smax, srow[j]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+            uint64_t U = 0;
+            for (int j = lane; j < nb; j += 32) U += mass_of(srow[j], smax);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) U += shfl_u64(U, lane ^ o);
+            const double thr = static_cast<double>(prm.p) * static_cast<double>(U);
+            uint64_t prefix = 0, above = 0;
+            bool done = false;
+            for (int pass = 0; pass < 6 && !done; ++pass) {
+                const int shift = 40 - 8 * pass;
+                for (int e = lane; e < 256; e += 32) {
+                    hm[e] = 0;
+                    hc[e] = 0;
+                }
+                __syncwarp();
+                for (int j = lane; j < nb; j += 32) {
+                    const uint64_t key = (static_cast<uint64_t>(order_key(srow[j])) << 16) |
+                                         static_cast<uint64_t>(0xFFFFu - j);
+                    if (pass == 0 || (key >> (shift + 8)) == prefix) {
+                        const int dg = static_cast<int>((key >> shift) & 255u);
+                        atomicAdd(reinterpret_cast<unsigned long long *>(&hm[dg]),
+                                  static_cast<unsigned long long>(mass_of(srow[j], smax)));
+                        atomicAdd(&hc[dg], 1u);
+                    }
+                }
+                __syncwarp();
+                // lane l owns digits 255-8l .. 248-8l (descending order)
+                uint64_t m8[8];
+                uint64_t tot = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    m8[e] = hm[255 - 8 * lane - e];
+                    tot += m8[e];
+                }
+                uint64_t incl = tot;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint64_t t = shfl_up_u64(incl, o);
+                    if (lane >= o) incl += t;
+                }
+                const uint64_t excl = incl - tot;
+                // first lane whose inclusive total reaches the threshold
+                const bool reach = static_cast<double>(above + incl) >= thr;
+                const unsigned ball = __ballot_sync(0xffffffffu, reach);
+                const int owner = __ffs(ball) - 1;  // always >= 0 (see invariant)
+                int digit = 0;
+                uint64_t new_above = 0;
+                uint32_t dcount = 0;
+                if (lane == owner) {
+                    uint64_t run = above + excl;
+                    int e = 0;
+                    for (; e < 8; ++e) {
+                        if (static_cast<double>(run + m8[e]) >= thr) break;
+                        run += m8[e];
+                    }
+                    digit = 255 - 8 * lane - e;
+                    new_above = run;
+                    dcount = hc[digit];
+                }
+                digit = __shfl_sync(0xffffffffu, digit, owner);
+                above = shfl_u64(new_above, owner);
+                dcount = __shfl_sync(0xffffffffu, dcount, owner);
+                prefix = (prefix << 8) | static_cast<uint64_t>(digit);
+                if (dcount == 1 || shift == 0) {
+                    cstar = prefix << shift;
+                    done = true;
+                }
+                __syncwarp();
+            }
+        }
+        // emit: bit row + ascending list
+        const int ti = i / (prm.Hp * prm.Wp), hi = (i / prm.Wp) % prm.Hp, wi = i % prm.Wp;
+        int cnt = 0;
+        uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
+        for (int w = 0; w < words; ++w) {
+            const int j = w * 32 + lane;
+            bool m = false;
+            if (j < nb) {
+                if (keep_all) {
+                    m = true;
+                } else if (!keep_none) {
+                    const uint64_t key = (static_cast<uint64_t>(order_key(srow[j])) << 16) |
+                                         static_cast<uint64_t>(0xFFFFu - j);
+                    m = key >= cstar;
+                }
+                m = m || (j == i);
+                if (!m && !(prm.flags & 1u)) {
+                    if (prm.flags & 2u) {
+                        m = true;
+                    } else {
+                        const int tj = j / (prm.Hp * prm.Wp), hj = (j / prm.Wp) % prm.Hp,
+                                  wj = j % prm.Wp;
+                        m = abs(ti - tj) <= prm.wt / 2 && abs(hi - hj) <= prm.wh / 2 &&
+                            abs(wi - wj) <= prm.ww / 2;
+                    }
+                }
+            }
+            const unsigned ball = __ballot_sync(0xffffffffu, m);
+            if (lane == 0) bits[(bh * nb + i) * words + w] = ball;
+            if (m) lst[cnt + __popc(ball & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+            cnt += __popc(ball);
+        }
+        if (lane == 0) row_cnt[bh * nb + i] = cnt;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// column lists: transpose of the bit rows.  One warp per (bh, 32-column word).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) col_lists_kernel(const uint32_t *__restrict__ bits,
+                                                        uint16_t *__restrict__ col_idx,
+                                                        int32_t *__restrict__ col_cnt,
+                                                        int64_t BH, int nb) {
+    const int words = (nb + 31) >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (gw >= BH * words) return;
+    const int64_t bh = gw / words;
+    const int w = static_cast<int>(gw % words);
+    const int j = w * 32 + lane;  // this lane's column
+    int cnt = 0;
+    uint16_t *lst = col_idx + (bh * nb + (j < nb ? j : 0)) * static_cast<int64_t>(nb);
+    for (int i0 = 0; i0 < nb; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t word = (i < nb) ? bits[(bh * nb + i) * words + w] : 0u;
+        uint32_t mine = 0;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+            const uint32_t col = __ballot_sync(0xffffffffu, (word >> c) & 1u);
+            if (lane == c) mine = col;
+        }
+        if (j < nb) {
+            while (mine) {
+                const int b = __ffs(mine) - 1;
+                mine &= mine - 1;
+                lst[cnt++] = static_cast<uint16_t>(i0 + b);
+            }
+        }
+    }
+    if (j < nb) col_cnt[bh * nb + j] = cnt;
+}
+
+}  // namespace nabla
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+size_t nabla_score_cut_smem(int nb, int D) {
+    const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
+    const size_t phase1 = sizeof(float) * (static_cast<size_t>(D) * nabla::kRows +
+                                           nabla::kDc * nabla::kCols);
+    const size_t phase2 = 8 * 256 * (sizeof(uint64_t) + sizeof(uint32_t));
+    return sizeof(float) * nabla::kRows * nbp + (phase1 > phase2 ? phase1 : phase2);
+}
+
+cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, float p,
+                                    float scale, int wt, int wh, int ww, unsigned flags,
+                                    const void *q, const void *k, float *qbar, float *kbar_t,
+                                    uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
+                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream) {
+    using namespace nabla;
+    const int bpc = 256 / (D / 8);
+    const int64_t tiles = (nb + bpc - 1) / bpc;
+    const dim3 pool_grid(static_cast<unsigned>(2 * BH * tiles));
+    if (D == 128)
+        pool_kernel<128><<<pool_grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
+            kbar_t, BH, nb);
+    else
+        pool_kernel<64><<<pool_grid, 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
+            kbar_t, BH, nb);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+
+    CutParams prm{nb, Hp, Wp, wt, wh, ww, flags, p, scale};
+    const size_t smem = nabla_score_cut_smem(nb, D);
+    const dim3 grid(static_cast<unsigned>(BH * ((nb + kRows - 1) / kRows)));
+    if (D == 128) {
+        err = cudaFuncSetAttribute(score_cut_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        score_cut_kernel<128><<<grid, kThreads, smem, stream>>>(qbar, kbar_t, prm, bits, row_idx,
+                                                                row_cnt);
+    } else {
+        err = cudaFuncSetAttribute(score_cut_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem));
+        if (err != cudaSuccess) return err;
+        score_cut_kernel<64><<<grid, kThreads, smem, stream>>>(qbar, kbar_t, prm, bits, row_idx,
+                                                               row_cnt);
+    }
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    if (col_idx) {
+        const int64_t warps = BH * ((nb + 31) / 32);
+        col_lists_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(
+            bits, col_idx, col_cnt, BH, nb);
+        err = cudaGetLastError();
+    }
+    return err;
+}

@@ -106,3 +106,28 @@ def bits(t: torch.Tensor):
     """Raw uint16 bits of a bf16 tensor as a numpy array (same shape)."""
     import numpy as np
     return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def make_inputs_device(w: Workload, seed0: int = 0, device="cuda", with_dout=None,
+                       rank: int = 0):
+    """Same recipe as make_inputs, drawn with a CUDA generator directly on the
+    device (fast for the benchmark's full-size workloads; the values differ
+    from the CPU stream).  Q, K, V in grid order [B*h, T*H*W, D], dout in
+    flattened order [B*h, N, D]; `rank` offsets the seeds."""
+    g = torch.Generator(device=device)
+    out = {}
+    ct, cy, cx = w.cell
+    nct, ncy, ncx = -(-w.T // ct), -(-w.H // cy), -(-w.W // cx)
+    for name, off in (("q", 1), ("k", 2), ("v", 3)):
+        g.manual_seed(int(seed0 + off + 1000 * rank))
+        c = torch.randn(w.BH, nct, ncy, ncx, w.D, generator=g, device=device)
+        c = (c.repeat_interleave(ct, 1).repeat_interleave(cy, 2).repeat_interleave(cx, 3)
+             [:, :w.T, :w.H, :w.W])
+        x = torch.randn(w.BH, w.T, w.H, w.W, w.D, generator=g, device=device)
+        x.mul_(w.noise).add_(c)
+        out[name] = x.to(torch.bfloat16).reshape(w.BH, w.N, w.D)
+        del c, x
+    if with_dout or (with_dout is None and w.backward):
+        g.manual_seed(int(seed0 + 4 + 1000 * rank))
+        out["dout"] = torch.randn(w.BH, w.N, w.D, generator=g, device=device).to(torch.bfloat16)
+    return out

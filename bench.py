@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the NABLA block-sparse attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input at
+the 720p-like training shape (B=1, 40 heads, 20 x 48 x 80 latent = 76,800
+tokens, head dim 128, p = 0.7, STA 3x3x3):
+    flatten Q, K, V (grid -> flattened order)
+    build the block mask (pool, pooled scores, CDF cut, STA, row + column lists)
+    block-sparse attention forward (O, LSE)
+    block-sparse attention backward (dQ, dK, dV)
+    unflatten O, dQ, dK, dV (flattened -> grid order)
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl nabla|reference]
+
+Prints one JSON line (rank 0).  `value` is effective TFLOP/s on kept blocks
+(forward 4*64*64*D + backward 10*64*64*D FLOP per kept block pair), whole job.
+Timing: CUDA events on the launching stream, barrier + synchronize around the
+K timed steps, max over ranks.  Every input tensor (786 MB) is larger than the
+126 MB L2, so no flush is needed between steps.
+"""
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse attn fwd/bwd ms & eff. TFLOP/s at 76.8K tokens; mask-build GB/s"
+WORKLOAD = "train"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("nabla", "reference"), default="nabla")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_config(w):
+    return {
+        "workload": "train-720p: B=%d heads=%d T*H*W=%dx%dx%d (%d tokens, %d blocks of 64) D=%d "
+                    "p=%.2f STA %dx%dx%d; flatten + mask + fwd + bwd + unflatten"
+                    % (w.B, w.heads, w.T, w.H, w.W, w.N, w.nb, w.D, w.p, *w.window),
+        "global_batch": w.B,
+        "seq_len": w.N,
+        "heads": w.heads,
+        "head_dim": w.D,
+        "p": w.p,
+        "sta_window": list(w.window),
+        "cell": list(w.cell),
+        "l2": "no flush: every input tensor (%.0f MB) exceeds the 126 MB L2" % (w.BH * w.N * w.D * 2 / 1e6),
+    }
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class Clocks:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# --------------------------------------------------------------------------
+def oracle_sample(w, n_blocks=24, seed=0):
+    """Oracle on one head of the workload: its mask (all rows) and the forward
+    on n_blocks sampled query blocks.  Returns (kept fwd FLOP, fwd seconds,
+    mask seconds, cores, description)."""
+    import numpy as np
+    import oracle
+    from adaptive_block_sparse_fractal_b200 import synth
+    w1 = synth.Workload(w.name, 1, 1, w.T, w.H, w.W, w.D, w.cell, w.p, w.window)
+    inp = synth.make_inputs(w1, seed, with_dout=False)
+    flat = {n: oracle.flatten_tokens(synth.bits(inp[n]).reshape(1, w.N, w.D), w.T, w.H, w.W, w.P)
+            for n in ("q", "k", "v")}
+    t0 = time.perf_counter()
+    m = oracle.build_mask(flat["q"], flat["k"], w.grid_blocks, w.p, w.scale, w.window, cols=False)
+    t_mask = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    sel = [(0, int(i)) for i in rng.choice(w.nb, n_blocks, replace=False)]
+    q, k, v = (oracle.bf16_bits_to_f64(flat[n]) for n in ("q", "k", "v"))
+    t0 = time.perf_counter()
+    oracle.attn_fwd(q, k, v, m["row_idx"], m["row_cnt"], w.scale, sel=sel)
+    t_fwd = time.perf_counter() - t0
+    kept = sum(int(m["row_cnt"][0, i]) for _, i in sel)
+    flop = 4.0 * 64 * 64 * w.D * kept
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    desc = ("oracle (float64 C, OpenMP) on one head of the same workload: mask build for all "
+            "%d rows (%.2f s) + forward on %d sampled query blocks (%d kept block pairs); value "
+            "= kept forward FLOP / forward seconds" % (w.nb, t_mask, n_blocks, kept))
+    return flop, t_fwd, t_mask, cores, desc
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing
+# --------------------------------------------------------------------------
+def dist_init(n):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d" % (n, world))
+    return rank, world, local
+
+
+def run_reference(args):
+    rank, world, _ = dist_init(args.gpus)
+    if rank != 0:
+        return 0
+    from adaptive_block_sparse_fractal_b200 import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    times, flops = [], []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        flop, t_fwd, t_mask, cores, desc = oracle_sample(w, n_blocks=8, seed=s)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(t_fwd)
+            flops.append(flop)
+    value = sum(flops) / sum(times) / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": desc.replace("24 sampled", "8 sampled")},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_nabla(args):
+    import torch
+    import torch.distributed as dist
+    from adaptive_block_sparse_fractal_b200 import nabla, synth
+
+    rank, world, local = dist_init(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    nabla.lib()
+    w = synth.WORKLOADS[WORKLOAD]
+    shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
+    prm = nabla.params_of(w.p, w.window, D=w.D, flags=nabla.EMIT_COLS)
+
+    grid = synth.make_inputs_device(w, args.seed, dev, with_dout=True, rank=rank)
+    B = {
+        "flat": {n: torch.empty_like(grid[n]) for n in ("q", "k", "v")},
+        "o": torch.empty_like(grid["q"]),
+        "lse": torch.empty((w.BH, w.N), dtype=torch.float32, device=dev),
+        "dq": torch.empty_like(grid["q"]), "dk": torch.empty_like(grid["q"]),
+        "dv": torch.empty_like(grid["q"]),
+        "out": {n: torch.empty_like(grid["q"]) for n in ("o", "dq", "dk", "dv")},
+        "mask": nabla.alloc_mask(shape, dev, cols=True),
+        "ws_mask": nabla.workspace(shape, nabla.OP_BUILD_MASK, dev),
+        "ws_fwd": nabla.workspace(shape, nabla.OP_ATTN_FWD, dev),
+        "ws_bwd": nabla.workspace(shape, nabla.OP_ATTN_BWD, dev),
+    }
+    stream = torch.cuda.current_stream(dev)
+
+    def step(src, ev=None):
+        for n in ("q", "k", "v"):
+            nabla.flatten(src[n], w.T, w.H, w.W, w.P, out=B["flat"][n])
+        if ev: ev[1].record(stream)
+        nabla.build_mask(shape, prm, B["flat"]["q"], B["flat"]["k"], mask=B["mask"],
+                         ws=B["ws_mask"])
+        if ev: ev[2].record(stream)
+        nabla.attn_fwd(shape, prm, B["flat"]["q"], B["flat"]["k"], B["flat"]["v"], B["mask"],
+                       o=B["o"], lse=B["lse"], ws=B["ws_fwd"])
+        if ev: ev[3].record(stream)
+        nabla.attn_bwd(shape, prm, B["flat"]["q"], B["flat"]["k"], B["flat"]["v"], B["o"],
+                       src["dout"], B["lse"], B["mask"], dq=B["dq"], dk=B["dk"], dv=B["dv"],
+                       ws=B["ws_bwd"])
+        if ev: ev[4].record(stream)
+        for n in ("o", "dq", "dk", "dv"):
+            nabla.flatten(B[n], w.T, w.H, w.W, w.P, inverse=True, out=B["out"][n])
+
+    launches_per_step = 3 + 3 + 1 + 3 + 4  # flatten, pool/score_cut/cols, fwd, bwd x3, unflatten
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step(grid)
+    barrier()
+    kept = int(B["mask"]["row_cnt"].sum().item())
+    kept_frac = kept / (w.BH * w.nb * w.nb)
+
+    # ---- device-resident timed region
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(args.steps):
+        evs[s][0].record(stream)
+        step(grid, evs[s])
+        evs[s][5].record(stream)
+    stop.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(start.elapsed_time(stop))
+    phase = [0.0] * 5
+    for s in range(args.steps):
+        for p in range(5):
+            phase[p] += evs[s][p].elapsed_time(evs[s][p + 1])
+    phase = [x / args.steps for x in phase]
+    ms_step = total_ms / args.steps
+
+    fwd_flop = 4.0 * 64 * 64 * w.D * kept
+    bwd_flop = 10.0 * 64 * 64 * w.D * kept
+    value = world * (fwd_flop + bwd_flop) / (ms_step * 1e-3) / 1e12
+    N, D, BH, nb = w.N, w.D, w.BH, w.nb
+    mask_bytes = (4.0 * N * D * BH + 16.0 * nb * D * BH + nb * nb * BH / 8.0
+                  + 2 * 2.0 * kept + 2 * 4.0 * BH * nb)
+    mask_gbs = mask_bytes / (phase[1] * 1e-3) / 1e9
+    flat_gbs = 3 * 2.0 * BH * N * D * 2 / (phase[0] * 1e-3) / 1e9
+
+    pk, pk_src = peaks()
+    ops = {"attn_bwd": (phase[3], bwd_flop), "attn_fwd": (phase[2], fwd_flop)}
+    dom = max(ops, key=lambda k: ops[k][0])
+    achieved = ops[dom][1] / (ops[dom][0] * 1e-3) / 1e12
+    peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "kernel": dom,
+                "peak_source": "bf16 sustained (of %s)" % pk_src,
+                "flop_per_launch": ops[dom][1], "ms_per_launch": ops[dom][0],
+                "frac_of_burst": achieved / pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])}
+
+    # ---- end to end through the C ABI with host buffers (pinned)
+    e2e = None
+    if not args.no_e2e:
+        host_in = {n: torch.empty(grid[n].shape, dtype=grid[n].dtype, pin_memory=True)
+                   for n in ("q", "k", "v", "dout")}
+        for n in host_in:
+            host_in[n].copy_(grid[n])
+        host_out = {n: torch.empty(grid["q"].shape, dtype=torch.bfloat16, pin_memory=True)
+                    for n in ("o", "dq", "dk", "dv")}
+        dev_in = grid  # device buffers refilled from the host every step
+
+        def e2e_step():
+            for n in host_in:
+                dev_in[n].copy_(host_in[n], non_blocking=True)
+            step(dev_in)
+            for n in host_out:
+                host_out[n].copy_(B["out"][n], non_blocking=True)
+
+        for _ in range(max(1, args.warmup // 2)):
+            e2e_step()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(a.elapsed_time(b)) / args.steps
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        e2e = {"value": world * (fwd_flop + bwd_flop) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        flop, t_fwd, t_mask, cores, desc = oracle_sample(w)
+        cpu = {"value": flop / t_fwd / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded cell-correlated bf16 Q/K/V (cell 2x8x8, noise 0.5), dO ~ "
+                    "N(0,1); each rank its own batch",
+            "config": workload_config(w),
+            "breakdown_ms": {"flatten_qkv": phase[0], "build_mask": phase[1],
+                             "attn_fwd": phase[2], "attn_bwd": phase[3],
+                             "unflatten_out": phase[4]},
+            "kept_blocks": kept, "kept_fraction": kept_frac,
+            "attn_fwd_tflops": fwd_flop / (phase[2] * 1e-3) / 1e12,
+            "attn_bwd_tflops": bwd_flop / (phase[3] * 1e-3) / 1e12,
+            "mask_build_gbs": mask_gbs, "mask_build_frac_hbm": mask_gbs / pk["hbm_gbs"],
+            "flatten_gbs": flat_gbs,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "gpu_launches": launches_per_step * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+    B.clear()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_nabla(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

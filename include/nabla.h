@@ -1,0 +1,186 @@
+/*
+ * nabla.h -- C ABI of libnabla.so: NABLA block-sparse 3D self-attention for
+ * video diffusion transformers, on NVIDIA B200 (sm_100a).
+ *
+ * The method is the one described in "NABLA: Neighborhood Adaptive Block-Level
+ * Attention" (gist.science technical summary, section 手法: NABLA):
+ *   1. fractal flattening of the T x H x W token grid (P x P patches made
+ *      contiguous, time order kept)                      -> nabla_flatten
+ *   2. mean-pooling Q and K into blocks of P*P tokens, the full attention map
+ *      over the pooled blocks, a per-row CDF cut at mass p, OR with a static
+ *      Sliding-Tile window (M = M_nabla OR M_STA)           -> nabla_build_mask
+ *   3. attention computed exactly on the kept blocks     -> nabla_attn_fwd
+ *   4. its gradients for training                        -> nabla_attn_bwd
+ *
+ * Conventions shared by every call
+ *   - All tensors live in device memory that the CALLER allocated; the library
+ *     allocates nothing and keeps no state between calls.  Scratch memory is
+ *     the caller's workspace, sized by nabla_workspace_size().
+ *   - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and returns without synchronising the host.
+ *     Errors found on the host (shape, alignment, parameters, workspace size,
+ *     launch failure) are returned immediately and nothing is enqueued.
+ *     A device-side failure (a bounded wait that expired) is written to the
+ *     status word at the start of the workspace; read it with nabla_status().
+ *   - Q, K, V, O, dO, dQ, dK, dV are bf16 (raw 16-bit patterns, nabla_bf16),
+ *     contiguous [B, heads, N, D] with N = T*H*W tokens in FLATTENED order.
+ *   - Pointers to tensors must be 16-byte aligned (NABLA_ERR_ALIGN).
+ *   - Supported: P = 8 (blocks of 64 tokens), D in {64, 128}, H and W
+ *     multiples of P, 1 <= number of blocks nb = T*(H/P)*(W/P) <= 2048.
+ *
+ * Return value of every int function: NABLA_OK (0) or a negative status.
+ */
+#ifndef NABLA_H
+#define NABLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t nabla_bf16;               /* raw bf16 bit pattern */
+typedef struct CUstream_st *nabla_stream_t; /* == cudaStream_t */
+
+#define NABLA_OK 0
+#define NABLA_ERR_SHAPE (-1)     /* grid not divisible by P, unsupported D, P or nb */
+#define NABLA_ERR_ALIGN (-2)     /* pointer not 16-byte aligned, inner_bytes % 16 != 0 */
+#define NABLA_ERR_PARAM (-3)     /* p not in [0,1], STA window even or < 1, scale <= 0 */
+#define NABLA_ERR_WORKSPACE (-4) /* workspace missing or smaller than required */
+#define NABLA_ERR_CUDA (-5)      /* a CUDA call or kernel launch failed */
+#define NABLA_ERR_TIMEOUT (-6)   /* a device-side bounded wait expired */
+#define NABLA_ERR_NULL (-7)      /* a required pointer is NULL */
+
+/* nabla_params.flags */
+#define NABLA_NO_STA 1u    /* no STA term: M = adaptive OR diagonal            */
+#define NABLA_FULL_STA 2u  /* STA window covers every block: dense attention   */
+#define NABLA_EMIT_COLS 4u /* also write the column lists needed by the backward */
+
+/* Problem shape.  P must be 8. */
+typedef struct {
+    int B, heads, T, H, W, D, P;
+} nabla_shape;
+
+/* Mask / attention parameters.
+ *   p      CDF mass threshold in [0, 1] ("thr" on the page).  Per row, the
+ *          kept adaptive set is the shortest run of blocks, taken in
+ *          descending pooled score (equal scores: lower index first), whose
+ *          softmax mass reaches p; p = 1 keeps every block, p = 0 none.
+ *   sta_t, sta_h, sta_w  odd STA window, in blocks (frames, patch rows,
+ *          patch columns), centred, truncated at the grid border.
+ *   scale  softmax scale of both the pooled map and the attention
+ *          (usually 1/sqrt(D)).
+ *   flags  NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS. */
+typedef struct {
+    float p;
+    int sta_t, sta_h, sta_w;
+    float scale;
+    unsigned flags;
+} nabla_params;
+
+/* Block mask M, caller-allocated (sizes from nabla_mask_bytes), device memory.
+ *   bits    [B*heads, nb, ceil(nb/32)] uint32: bit (j % 32) of word j / 32 of
+ *           row i is set when block j is kept for query block i.
+ *   row_idx [B*heads, nb, nb] uint16: kept j of row i, ascending; only the
+ *           first row_cnt entries of each row are written.
+ *   row_cnt [B*heads, nb] int32.
+ *   col_idx, col_cnt: the transpose (query blocks i keeping key block j,
+ *           ascending i); written only with NABLA_EMIT_COLS, required by
+ *           nabla_attn_bwd.  May be NULL otherwise. */
+typedef struct {
+    uint32_t *bits;
+    uint16_t *row_idx;
+    int32_t *row_cnt;
+    uint16_t *col_idx;
+    int32_t *col_cnt;
+} nabla_mask;
+
+/* Which part of the mask nabla_mask_bytes() sizes. */
+#define NABLA_MASK_BITS 0
+#define NABLA_MASK_ROW_IDX 1
+#define NABLA_MASK_ROW_CNT 2
+#define NABLA_MASK_COL_IDX 3
+#define NABLA_MASK_COL_CNT 4
+
+/* Which call nabla_workspace_size() sizes. */
+#define NABLA_OP_BUILD_MASK 0
+#define NABLA_OP_ATTN_FWD 1
+#define NABLA_OP_ATTN_BWD 2
+
+/* Fractal flattening (section 手法: NABLA, "トークン再順序付け (Fractal
+ * Flattening)").  `in` and `out` are [outer, T, H, W, inner_bytes] in grid
+ * order and [outer, N, inner_bytes] in flattened order, where token (t, y, x)
+ * goes to
+ *   n = ((t*(H/P) + y/P)*(W/P) + x/P)*P*P + (y%P)*P + x%P
+ * (one level of P x P patches, patch grid and patch interior row-major).
+ * inverse = 0 maps grid -> flattened, inverse = 1 flattened -> grid.
+ * Any P >= 1 dividing H and W; inner_bytes % 16 == 0; in != out (no
+ * in-place).  Works for [B, T, H, W, C] activations and [B*h, T, H, W, D]
+ * heads alike. */
+int nabla_flatten(const void *in, void *out, int64_t outer, int T, int H, int W, int P,
+                  int64_t inner_bytes, int inverse, nabla_stream_t stream);
+
+/* Bytes of workspace `op` needs for `shape` (0 for an invalid shape).
+ * Every workspace starts with a 256-byte status region. */
+size_t nabla_workspace_size(const nabla_shape *shape, int op);
+
+/* Bytes of mask part `part` (NABLA_MASK_*) for `shape` (0 if invalid). */
+size_t nabla_mask_bytes(const nabla_shape *shape, int part);
+
+/* Build M from flattened q, k (section 手法: NABLA, "適応型マスク構築" and
+ * "STA とのハイブリッド統合").  Per (batch, head) and query block i:
+ *   qbar_i, kbar_j = means of the 64 tokens of block i / j, summed in float32
+ *                    in ascending token order, times 1/64;
+ *   s_ij           = float32 fused multiply-add chain over d ascending, times
+ *                    scale;
+ *   w_ij           = exp(s_ij - max_j s_ij) in float64, mass u_ij =
+ *                    floor(w_ij * 2^40) as an exact integer;
+ *   adaptive set   = shortest prefix of j ordered by (s_ij desc, j asc) whose
+ *                    summed u reaches p * sum_j u_ij (float64 product);
+ *   M_ij           = adaptive OR STA window OR (i == j).
+ * Writes bits, row lists, and (with NABLA_EMIT_COLS) column lists.
+ * Workspace: nabla_workspace_size(shape, NABLA_OP_BUILD_MASK) bytes, 256-byte
+ * aligned. */
+int nabla_build_mask(const nabla_shape *shape, const nabla_params *params,
+                     const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
+                     void *workspace, size_t workspace_bytes, nabla_stream_t stream);
+
+/* Block-sparse attention forward over M (bullet "拡張": attention is
+ * computed for the kept blocks only).  For query token n of block i:
+ *   o_n   = sum over tokens m of blocks j in row i of M of
+ *           softmax_m(scale * q_n . k_m) v_m          (bf16 out, fp32 accumulate)
+ *   lse_n = log sum_m exp(scale * q_n . k_m)          (float32 [B*heads, N])
+ * Needs mask->row_idx and mask->row_cnt.  lse may be NULL when no backward
+ * follows.  Workspace: nabla_workspace_size(shape, NABLA_OP_ATTN_FWD). */
+int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
+                   const nabla_bf16 *k, const nabla_bf16 *v, const nabla_mask *mask,
+                   nabla_bf16 *o, float *lse, void *workspace, size_t workspace_bytes,
+                   nabla_stream_t stream);
+
+/* Gradients of nabla_attn_fwd (training through NABLA):
+ *   D_n = dO_n . o_n,  P_nm = exp(scale q_n.k_m - lse_n),
+ *   dV_m = sum_n P_nm dO_n,  dS_nm = P_nm (dO_n . v_m - D_n),
+ *   dQ_n = scale sum_m dS_nm k_m,  dK_m = scale sum_n dS_nm q_n,
+ * over the pairs kept by M.  Needs row AND column lists (build the mask with
+ * NABLA_EMIT_COLS) and the o, lse written by nabla_attn_fwd.  Deterministic
+ * (no atomics).  Workspace: nabla_workspace_size(shape, NABLA_OP_ATTN_BWD). */
+int nabla_attn_bwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
+                   const nabla_bf16 *k, const nabla_bf16 *v, const nabla_bf16 *o,
+                   const nabla_bf16 *dout, const float *lse, const nabla_mask *mask,
+                   nabla_bf16 *dq, nabla_bf16 *dk, nabla_bf16 *dv, void *workspace,
+                   size_t workspace_bytes, nabla_stream_t stream);
+
+/* Synchronises `stream`, then returns the device-side status recorded in the
+ * workspace by the last call that used it (NABLA_OK or NABLA_ERR_TIMEOUT),
+ * or NABLA_ERR_CUDA if the stream reports an error. */
+int nabla_status(const void *workspace, nabla_stream_t stream);
+
+/* Static string for a status code. */
+const char *nabla_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NABLA_H */

@@ -294,6 +294,10 @@ static int64_t cut_row_fixed(const float *score, int64_t nb, float p, uint8_t *k
         if (margin) *margin = INFINITY;
         return nb;
     }
+    if (p <= 0.0f) { /* the empty prefix already reaches 0: nothing to decide */
+        if (margin) *margin = INFINITY;
+        return 0;
+    }
     float smax = -INFINITY;
     for (int64_t j = 0; j < nb; ++j) smax = fmaxf(smax, score[j]);
     uint64_t U = 0;

@@ -1,0 +1,136 @@
+"""The C-ABI library without a GPU: it loads, exports every function that
+include/nabla.h declares, sizes buffers as documented, and rejects invalid
+arguments on the host before enqueuing anything (fault injection on the
+host: bad shapes, parameters, NULL and misaligned pointers, short
+workspaces)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from adaptive_block_sparse_fractal_b200 import build, nabla
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return nabla.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "nabla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return set(re.findall(r"\b(nabla_[a-z_]+)\s*\(", src))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared()
+    assert declared == set(nabla.SYMBOLS)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_strerror(L):
+    for st in (0, -1, -2, -3, -4, -5, -6, -7):
+        assert nabla.strerror(st) and nabla.strerror(st) != "unknown status"
+    assert nabla.strerror(-99) == "unknown status"
+
+
+def _shape(**kw):
+    d = dict(B=1, heads=40, T=20, H=48, W=80, D=128, P=8)
+    d.update(kw)
+    return nabla.Shape(*(d[k] for k in ("B", "heads", "T", "H", "W", "D", "P")))
+
+
+def test_sizes(L):
+    s = _shape()
+    BH, nb, N, D = 40, 1200, 76800, 128
+    assert nabla.mask_bytes(s, nabla.MASK_BITS) == BH * nb * ((nb + 31) // 32) * 4
+    assert nabla.mask_bytes(s, nabla.MASK_ROW_IDX) == BH * nb * nb * 2
+    assert nabla.mask_bytes(s, nabla.MASK_COL_CNT) == BH * nb * 4
+    assert nabla.workspace_size(s, nabla.OP_BUILD_MASK) == 256 + 2 * BH * nb * D * 4
+    assert nabla.workspace_size(s, nabla.OP_ATTN_BWD) == 256 + BH * N * 4
+    assert nabla.workspace_size(s, nabla.OP_ATTN_FWD) >= 256
+    # invalid shapes size to 0
+    for bad in (_shape(P=4), _shape(D=96), _shape(H=50), _shape(T=0), _shape(T=200)):
+        assert nabla.workspace_size(bad, nabla.OP_BUILD_MASK) == 0
+        assert nabla.mask_bytes(bad, nabla.MASK_BITS) == 0
+
+
+FAKE = ctypes.c_void_p(0x10000)  # never dereferenced: every call below fails validation
+FAKE_ODD = ctypes.c_void_p(0x10008)
+
+
+def _mask():
+    return nabla.MaskStruct(FAKE, FAKE, FAKE, FAKE, FAKE)
+
+
+def _build(L, shape, params, q=FAKE, k=FAKE, mask=None, ws=FAKE, ws_bytes=1 << 40):
+    m = _mask() if mask is None else mask
+    return L.nabla_build_mask(ctypes.byref(shape), ctypes.byref(params), q, k, ctypes.byref(m),
+                              ws, ws_bytes, None)
+
+
+def test_build_mask_rejects_on_host(L):
+    good = nabla.params_of(0.7, (3, 3, 3), D=128)
+    assert _build(L, _shape(H=44), good) == nabla.ERR_SHAPE
+    assert _build(L, _shape(D=32), good) == nabla.ERR_SHAPE
+    for p in (-0.1, 1.5, float("nan")):
+        assert _build(L, _shape(), nabla.params_of(p, (3, 3, 3), D=128)) == nabla.ERR_PARAM
+    assert _build(L, _shape(), nabla.params_of(0.5, (2, 3, 3), D=128)) == nabla.ERR_PARAM
+    assert _build(L, _shape(), nabla.params_of(0.5, (3, 3, 0), D=128)) == nabla.ERR_PARAM
+    assert _build(L, _shape(), nabla.params_of(0.5, (3, 3, 3), scale=0.0)) == nabla.ERR_PARAM
+    both = nabla.params_of(0.5, (3, 3, 3), D=128, flags=nabla.NO_STA | nabla.FULL_STA)
+    assert _build(L, _shape(), both) == nabla.ERR_PARAM
+    # even windows are fine when the STA term is off
+    nosta = nabla.params_of(0.5, (2, 2, 2), D=128, flags=nabla.NO_STA)
+    assert _build(L, _shape(), nosta, q=None) == nabla.ERR_NULL
+    assert _build(L, _shape(), good, k=None) == nabla.ERR_NULL
+    cols = nabla.params_of(0.5, (3, 3, 3), D=128, flags=nabla.EMIT_COLS)
+    assert _build(L, _shape(), cols, mask=nabla.MaskStruct(FAKE, FAKE, FAKE, None, None)) == \
+        nabla.ERR_NULL
+    assert _build(L, _shape(), good, q=FAKE_ODD) == nabla.ERR_ALIGN
+    assert _build(L, _shape(), good, ws=None) == nabla.ERR_WORKSPACE
+    assert _build(L, _shape(), good, ws_bytes=1024) == nabla.ERR_WORKSPACE
+    assert _build(L, _shape(), good, ws=FAKE_ODD) == nabla.ERR_ALIGN
+    assert L.nabla_build_mask(None, ctypes.byref(good), FAKE, FAKE, ctypes.byref(_mask()), FAKE,
+                              1 << 40, None) == nabla.ERR_NULL
+
+
+def test_attention_rejects_on_host(L):
+    s, good = _shape(), nabla.params_of(0.7, (3, 3, 3), D=128)
+    m = _mask()
+    fwd = lambda *a: L.nabla_attn_fwd(ctypes.byref(s), ctypes.byref(good), *a)
+    assert fwd(FAKE, FAKE, None, ctypes.byref(m), FAKE, None, FAKE, 1 << 40, None) == nabla.ERR_NULL
+    assert fwd(FAKE, FAKE_ODD, FAKE, ctypes.byref(m), FAKE, None, FAKE, 1 << 40, None) == \
+        nabla.ERR_ALIGN
+    assert fwd(FAKE, FAKE, FAKE, ctypes.byref(m), FAKE, None, FAKE, 16, None) == \
+        nabla.ERR_WORKSPACE
+    nocols = nabla.MaskStruct(FAKE, FAKE, FAKE, None, None)
+    bwd = lambda mask, ws_bytes: L.nabla_attn_bwd(
+        ctypes.byref(s), ctypes.byref(good), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+        ctypes.byref(mask), FAKE, FAKE, FAKE, FAKE, ws_bytes, None)
+    assert bwd(nocols, 1 << 40) == nabla.ERR_NULL  # backward needs column lists
+    assert bwd(m, 1024) == nabla.ERR_WORKSPACE
+
+
+def test_flatten_rejects_on_host(L):
+    f = L.nabla_flatten
+    assert f(None, FAKE, 1, 2, 16, 16, 8, 256, 0, None) == nabla.ERR_NULL
+    assert f(None, None, 0, 2, 16, 16, 8, 256, 0, None) == nabla.OK  # empty: nothing to touch
+    assert f(FAKE, FAKE_ODD, 1, 2, 16, 16, 8, 256, 0, None) == nabla.ERR_ALIGN
+    assert f(FAKE, ctypes.c_void_p(0x20000), 1, 2, 16, 16, 8, 24, 0, None) == nabla.ERR_ALIGN
+    assert f(FAKE, ctypes.c_void_p(0x20000), 1, 2, 16, 12, 8, 256, 0, None) == nabla.ERR_SHAPE
+    assert f(FAKE, FAKE, 1, 2, 16, 16, 8, 256, 0, None) == nabla.ERR_PARAM  # in place
+    # empty inputs are a successful no-op
+    assert f(FAKE, ctypes.c_void_p(0x20000), 0, 2, 16, 16, 8, 256, 0, None) == nabla.OK
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(nabla, "_lib", None)
+    monkeypatch.setattr(nabla, "LIB_PATH", "/nonexistent/libnabla.so")
+    with pytest.raises(RuntimeError, match="not built"):
+        nabla.lib()
