@@ -3,6 +3,7 @@
 // error is returned before anything is enqueued.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/nabla.h"
 #include "common.cuh"
@@ -232,3 +233,66 @@ const char *nabla_strerror(int status) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// nabla_build_mask_static: the mask build with its scratch (the pooled means)
+// in an array compiled into this library instead of a caller workspace.  For
+// callers that are handed only their input and output buffers and may not
+// call cudaMalloc themselves.  The array is allocated once per GPU when the
+// library's device code is loaded there and held until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_mask_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+void *g_scratch_addr[kMaxDevices];  // device address of g_mask_scratch, per device
+std::mutex g_scratch_mutex;
+
+// Device address of the scratch array on the current device.  The first call
+// on a device looks it up (the host-side name is only a stand-in, never a
+// device address) and caches it.
+int static_scratch(void **addr) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NABLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (g_scratch_addr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_mask_scratch) != cudaSuccess || p == nullptr)
+            return NABLA_ERR_CUDA;
+        g_scratch_addr[dev] = p;
+    }
+    *addr = g_scratch_addr[dev];
+    return NABLA_OK;
+}
+
+}  // namespace
+
+extern "C" int nabla_build_mask_static(const nabla_shape *shape, const nabla_params *params,
+                                       const nabla_bf16 *q, const nabla_bf16 *k,
+                                       const nabla_mask *mask, nabla_stream_t stream) {
+    Dims d;
+    int st = check_shape(shape, &d);
+    if (st != NABLA_OK) return st;
+    if ((st = check_params(params, true)) != NABLA_OK) return st;
+    if (q == nullptr || k == nullptr || mask == nullptr || mask->bits == nullptr ||
+        mask->row_idx == nullptr || mask->row_cnt == nullptr)
+        return NABLA_ERR_NULL;
+    const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
+    if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k)) return NABLA_ERR_ALIGN;
+    const size_t half = round256(sizeof(float) * d.BH * d.nb * d.D);
+    if (2 * half > kStaticScratchBytes) return NABLA_ERR_WORKSPACE;
+    void *base = nullptr;
+    if ((st = static_scratch(&base)) != NABLA_OK) return st;
+    // Every byte of the scratch that this call reads is written earlier in the
+    // same call (pool kernel), so nothing has to be cleared first.
+    float *qbar = static_cast<float *>(base);
+    float *kbar_t = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + half);
+    return cuda_status(nabla_launch_build_mask(
+        d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
+        params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
+        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr,
+        reinterpret_cast<cudaStream_t>(stream)));
+}

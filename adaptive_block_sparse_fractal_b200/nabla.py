@@ -21,7 +21,8 @@ MASK_BITS, MASK_ROW_IDX, MASK_ROW_CNT, MASK_COL_IDX, MASK_COL_CNT = 0, 1, 2, 3, 
 
 # every symbol include/nabla.h declares
 SYMBOLS = ("nabla_flatten", "nabla_workspace_size", "nabla_mask_bytes", "nabla_build_mask",
-           "nabla_attn_fwd", "nabla_attn_bwd", "nabla_status", "nabla_strerror")
+           "nabla_build_mask_static", "nabla_attn_fwd", "nabla_attn_bwd", "nabla_status",
+           "nabla_strerror")
 
 
 class NablaError(RuntimeError):
@@ -63,6 +64,8 @@ def lib():
         L.nabla_mask_bytes.restype = SZ
         L.nabla_build_mask.argtypes = [P, P, P, P, P, P, SZ, P]
         L.nabla_build_mask.restype = I
+        L.nabla_build_mask_static.argtypes = [P, P, P, P, P, P]
+        L.nabla_build_mask_static.restype = I
         L.nabla_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, P, SZ, P]
         L.nabla_attn_fwd.restype = I
         L.nabla_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]

@@ -146,6 +146,31 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params,
                      const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
                      void *workspace, size_t workspace_bytes, nabla_stream_t stream);
 
+/* Same computation and outputs as nabla_build_mask, without a workspace.
+ * (No counterpart on the page: this is a calling convenience.)
+ *
+ * For callers that are handed only their input and output buffers and cannot
+ * call cudaMalloc -- for example a plugin interface that passes no workspace,
+ * or a process whose device memory is reserved up front by another allocator
+ * -- so cannot provide the scratch nabla_build_mask needs for the pooled
+ * means.  Here that scratch is a 32 MiB array compiled into the library: every
+ * GPU that loads the library holds those 32 MiB until the process exits.
+ *   - Limit: 2 * round_up_256(4 * B*heads * nb * D) <= 32 MiB (e.g. 16 heads of
+ *     a 1440-block, D = 128 problem fit; 40 heads of 1200 blocks do not).
+ *     Larger shapes return NABLA_ERR_WORKSPACE and enqueue nothing.
+ *   - The first call on a device (the current device) looks up the array's
+ *     device address with cudaGetSymbolAddress; make that first call before
+ *     any stream capture on that device.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *   - All calls share the one array per device, which keeps the last call's
+ *     contents.  Calls whose GPU work overlaps (other streams, other host
+ *     threads) race on it; serialise them.  Nothing in the array needs to
+ *     start at zero: each call writes every scratch byte it reads.
+ * Other arguments, checks and outputs: as nabla_build_mask. */
+int nabla_build_mask_static(const nabla_shape *shape, const nabla_params *params,
+                            const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
+                            nabla_stream_t stream);
+
 /* Block-sparse attention forward over M (bullet "拡張": attention is
  * computed for the kept blocks only).  For query token n of block i:
  *   o_n   = sum over tokens m of blocks j in row i of M of
