@@ -34,6 +34,12 @@ constexpr int kMaxNb = 2048;
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Scratch of the mask build: pooled Q [BH, nb, D] then pooled K transposed
+// [BH, D, nbp] (nbp = nb rounded up to a multiple of 4).
+struct MaskScratch {
+    size_t qbar_bytes, kbar_bytes;
+};
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct Dims {
@@ -70,10 +76,20 @@ int check_params(const nabla_params *p, bool need_window) {
     return NABLA_OK;
 }
 
+MaskScratch mask_scratch(const Dims &d) {
+    const size_t nbp = (static_cast<size_t>(d.nb) + 3) & ~static_cast<size_t>(3);
+    return {round256(sizeof(float) * d.BH * d.nb * d.D), round256(sizeof(float) * d.BH * d.D * nbp)};
+}
+
+size_t mask_scratch_bytes(const Dims &d) {
+    const MaskScratch m = mask_scratch(d);
+    return m.qbar_bytes + m.kbar_bytes;
+}
+
 size_t ws_bytes(const Dims &d, int op) {
     switch (op) {
         case NABLA_OP_BUILD_MASK:
-            return kStatusBytes + 2 * round256(sizeof(float) * d.BH * d.nb * d.D);
+            return kStatusBytes + mask_scratch_bytes(d);
         case NABLA_OP_ATTN_FWD:
             return kStatusBytes;
         case NABLA_OP_ATTN_BWD:
@@ -154,7 +170,7 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params, const
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
     unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
     float *qbar = reinterpret_cast<float *>(w);
-    float *kbar_t = reinterpret_cast<float *>(w + round256(sizeof(float) * d.BH * d.nb * d.D));
+    float *kbar_t = reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
         d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
         params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
@@ -282,14 +298,14 @@ extern "C" int nabla_build_mask_static(const nabla_shape *shape, const nabla_par
     const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
     if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k)) return NABLA_ERR_ALIGN;
-    const size_t half = round256(sizeof(float) * d.BH * d.nb * d.D);
-    if (2 * half > kStaticScratchBytes) return NABLA_ERR_WORKSPACE;
+    const MaskScratch ms = mask_scratch(d);
+    if (ms.qbar_bytes + ms.kbar_bytes > kStaticScratchBytes) return NABLA_ERR_WORKSPACE;
     void *base = nullptr;
     if ((st = static_scratch(&base)) != NABLA_OK) return st;
     // Every byte of the scratch that this call reads is written earlier in the
     // same call (pool kernel), so nothing has to be cleared first.
     float *qbar = static_cast<float *>(base);
-    float *kbar_t = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + half);
+    float *kbar_t = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + ms.qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
         d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
         params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,

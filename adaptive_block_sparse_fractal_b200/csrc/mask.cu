@@ -9,13 +9,14 @@
 //   score_cut_kernel   per (bh, 16 query blocks): pooled scores as a float32
 //                      fma chain over d ascending (register-tiled FFMA; the
 //                      order per output is the plain ascending chain), then
-//                      per row: weights exp(s - max) in float64, integer mass
-//                      floor(w * 2^40), a radix select over the 48-bit key
-//                      (score bits, then inverted block index) that finds the
-//                      last block of the shortest descending prefix whose mass
-//                      reaches p * total, and the OR with the STA window and
-//                      the diagonal.  Writes the bit row and the ascending row
-//                      list.
+//                      per row (one warp, values in registers): weights
+//                      exp(s - max) in float64, integer mass floor(w * 2^40),
+//                      a bitwise bisection over the 48-bit key (score bits,
+//                      then inverted block index, only when scores tie) for
+//                      the last block of the shortest descending prefix whose
+//                      mass reaches p * total, and the OR with the STA window
+//                      and the diagonal.  Writes the bit row and the ascending
+//                      row list.
 //   col_lists_kernel   transpose of the bit rows into ascending column lists.
 //
 // The mass sums are exact integers, so the selected set does not depend on
@@ -49,6 +50,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restri
     const int i = i0 + bl;
     const __nv_bfloat16 *x = which ? k : q;
     const int64_t N = static_cast<int64_t>(nb) * kBlk;
+    const int nbp = (nb + 3) & ~3;  // row stride of the transposed K-bar
 
     float acc[8];
 #pragma unroll
@@ -89,7 +91,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restri
         // write [D][nb]: each thread writes consecutive blocks of one feature
         for (int idx = tid; idx < D * BPC; idx += 256) {
             const int d = idx / BPC, b = idx % BPC;
-            if (i0 + b < nb) kbar_t[(bh * D + d) * nb + i0 + b] = tile[b][d];
+            if (i0 + b < nb) kbar_t[(bh * D + d) * nbp + i0 + b] = tile[b][d];
         }
     }
 }
@@ -114,23 +116,22 @@ __device__ __forceinline__ uint32_t order_key(float s) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-__device__ __forceinline__ uint64_t mass_of(float s, float smax) {
+// Integer mass floor(exp(s - smax) * 2^40), held in a double (exact: an
+// integer <= 2^40; sums of up to 2^13 of them stay below 2^53, so every sum
+// below is exact whatever the order of the additions).
+__device__ __forceinline__ double mass_of(float s, float smax) {
     const double w = exp(static_cast<double>(s) - static_cast<double>(smax));
-    return __double2ull_rz(w * 1099511627776.0);  // * 2^40, exact scaling
+    return trunc(w * 1099511627776.0);  // * 2^40 is an exact scaling
 }
 
-__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
-    uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v), src);
-    uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), src);
-    return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-__device__ __forceinline__ uint64_t shfl_up_u64(uint64_t v, int d) {
-    uint32_t lo = __shfl_up_sync(0xffffffffu, static_cast<uint32_t>(v), d);
-    uint32_t hi = __shfl_up_sync(0xffffffffu, static_cast<uint32_t>(v >> 32), d);
-    return (static_cast<uint64_t>(hi) << 32) | lo;
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
 }
 
-template <int D>
+// One warp per query row.  E = elements per lane (nb <= 32 * E).
+template <int D, int E>
 __global__ void __launch_bounds__(kThreads, 1)
     score_cut_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar_t,
                      CutParams prm, uint32_t *__restrict__ bits, uint16_t *__restrict__ row_idx,
@@ -139,11 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nb = prm.nb;
     const int nbp = (nb + 3) & ~3;
     float *sS = reinterpret_cast<float *>(smem);                       // [kRows][nbp]
-    unsigned char *work = smem + sizeof(float) * kRows * nbp;          // phase-specific
-    float *sQt = reinterpret_cast<float *>(work);                      // [D][kRows]
-    float *sKt = sQt + D * kRows;                                      // [kDc][kCols]
-    uint64_t *hmass = reinterpret_cast<uint64_t *>(work);              // [8 warps][256]
-    uint32_t *hcnt = reinterpret_cast<uint32_t *>(hmass + 8 * 256);    // [8 warps][256]
+    float *sQt = reinterpret_cast<float *>(smem + sizeof(float) * kRows * nbp);  // [D][kRows]
+    float *sKt = sQt + D * kRows;                                      // [2][kDc][kCols]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tiles = (nb + kRows - 1) / kRows;
@@ -151,51 +149,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i0 = (blockIdx.x % tiles) * kRows;
 
     // ---- phase 1: scores s[r][j] = (fma chain over d of qbar_i . kbar_j) * scale
+    // K-bar slices [kDc features][kCols blocks] stream through a double buffer
+    // with cp.async; the accumulation per output still runs d = 0, 1, ... D-1.
     for (int idx = tid; idx < kRows * D; idx += kThreads) {
         const int r = idx / D, d = idx % D;
         sQt[d * kRows + r] = (i0 + r < nb) ? qbar[(bh * nb + i0 + r) * D + d] : 0.f;
     }
     const int cg = tid % 64;  // 4 consecutive columns
     const int rg = tid / 64;  // 4 consecutive rows
-    const float *kt = kbar_t + bh * static_cast<int64_t>(D) * nb;
-    for (int j0 = 0; j0 < nb; j0 += kCols) {
-        float acc[4][4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-        for (int d0 = 0; d0 < D; d0 += kDc) {
-            __syncthreads();
-            for (int idx = tid; idx < kDc * kCols; idx += kThreads) {
-                const int d = idx / kCols, j = idx % kCols;
-                sKt[idx] = (j0 + j < nb) ? kt[static_cast<int64_t>(d0 + d) * nb + j0 + j] : 0.f;
-            }
-            __syncthreads();
-#pragma unroll 8
-            for (int d = 0; d < kDc; ++d) {
-                const float4 qv = *reinterpret_cast<const float4 *>(sQt + (d0 + d) * kRows + rg * 4);
-                const float4 kv = *reinterpret_cast<const float4 *>(sKt + d * kCols + cg * 4);
-                const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-                const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(qa[a], ka[b], acc[a][b]);
+    const float *kt = kbar_t + bh * static_cast<int64_t>(D) * nbp;
+    constexpr int DCH = D / kDc;  // feature slices per column tile
+    const int nstage = ((nb + kCols - 1) / kCols) * DCH;
+    auto issue = [&](int st) {
+        const int j0 = (st / DCH) * kCols, d0 = (st % DCH) * kDc;
+        float *dst = sKt + (st & 1) * (kDc * kCols);
+        // kDc rows of kCols floats = kDc * kCols / 4 chunks of 16 bytes
+        for (int c = tid; c < kDc * kCols / 4; c += kThreads) {
+            const int d = c / (kCols / 4), j = (c % (kCols / 4)) * 4;
+            float *sd = dst + d * kCols + j;
+            if (j0 + j < nbp) {
+                cp_async16(smem_addr(sd), kt + static_cast<int64_t>(d0 + d) * nbp + j0 + j);
+            } else {
+                sd[0] = sd[1] = sd[2] = sd[3] = 0.f;
             }
         }
+        cp_async_commit();
+    };
+    float acc[4][4];
+    issue(0);
+    for (int st = 0; st < nstage; ++st) {
+        if (st + 1 < nstage) {
+            issue(st + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const int j0 = (st / DCH) * kCols, d0 = (st % DCH) * kDc;
+        if (d0 == 0) {
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                const int j = j0 + cg * 4 + b;
-                if (j < nb) sS[(rg * 4 + a) * nbp + j] = __fmul_rn(acc[a][b], prm.scale);
-            }
+                for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+        }
+        const float *sk = sKt + (st & 1) * (kDc * kCols);
+#pragma unroll 8
+        for (int d = 0; d < kDc; ++d) {
+            const float4 qv = *reinterpret_cast<const float4 *>(sQt + (d0 + d) * kRows + rg * 4);
+            const float4 kv = *reinterpret_cast<const float4 *>(sk + d * kCols + cg * 4);
+            const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
+            const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(qa[a], ka[b], acc[a][b]);
+        }
+        if (d0 + kDc == D) {
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    const int j = j0 + cg * 4 + b;
+                    if (j < nb) sS[(rg * 4 + a) * nbp + j] = __fmul_rn(acc[a][b], prm.scale);
+                }
+        }
+        __syncthreads();
     }
-    __syncthreads();
 
-    // ---- phase 2: one warp per row
-    uint64_t *hm = hmass + warp * 256;
-    uint32_t *hc = hcnt + warp * 256;
+    // ---- phase 2: one warp per row; keys and masses in registers
     const int words = (nb + 31) >> 5;
     const bool keep_all = prm.p >= 1.0f;
     const bool keep_none = prm.p <= 0.0f;
@@ -203,80 +224,75 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i = i0 + r;
         if (i >= nb) break;
         const float *srow = sS + r * nbp;
-        uint64_t cstar = 0;  // composite key of the last kept block
+        uint64_t cstar = 0;  // composite key (score key, 0xFFFF - j) of the last kept block
         if (!keep_all && !keep_none) {
+            uint32_t kv[E];
+            double wv[E];
             float smax = -INFINITY;
-            for (int j = lane; j < nb; j += 32) smax = fmaxf(smax, srow[j]);
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int j = lane + 32 * e;
+                if (j < nb) smax = fmaxf(smax, srow[j]);
+            }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
-            uint64_t U = 0;
-            for (int j = lane; j < nb; j += 32) U += mass_of(srow[j], smax);
+            double U = 0.0;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) U += shfl_u64(U, lane ^ o);
-            const double thr = static_cast<double>(prm.p) * static_cast<double>(U);
-            uint64_t prefix = 0, above = 0;
-            bool done = false;
-            for (int pass = 0; pass < 6 && !done; ++pass) {
-                const int shift = 40 - 8 * pass;
-                for (int e = lane; e < 256; e += 32) {
-                    hm[e] = 0;
-                    hc[e] = 0;
-                }
-                __syncwarp();
-                for (int j = lane; j < nb; j += 32) {
-                    const uint64_t key = (static_cast<uint64_t>(order_key(srow[j])) << 16) |
-                                         static_cast<uint64_t>(0xFFFFu - j);
-                    if (pass == 0 || (key >> (shift + 8)) == prefix) {
-                        const int dg = static_cast<int>((key >> shift) & 255u);
-                        atomicAdd(reinterpret_cast<unsigned long long *>(&hm[dg]),
-                                  static_cast<unsigned long long>(mass_of(srow[j], smax)));
-                        atomicAdd(&hc[dg], 1u);
-                    }
-                }
-                __syncwarp();
-                // lane l owns digits 255-8l .. 248-8l (descending order)
-                uint64_t m8[8];
-                uint64_t tot = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    m8[e] = hm[255 - 8 * lane - e];
-                    tot += m8[e];
-                }
-                uint64_t incl = tot;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint64_t t = shfl_up_u64(incl, o);
-                    if (lane >= o) incl += t;
-                }
-                const uint64_t excl = incl - tot;
-                // first lane whose inclusive total reaches the threshold
-                const bool reach = static_cast<double>(above + incl) >= thr;
-                const unsigned ball = __ballot_sync(0xffffffffu, reach);
-                const int owner = __ffs(ball) - 1;  // always >= 0 (see invariant)
-                int digit = 0;
-                uint64_t new_above = 0;
-                uint32_t dcount = 0;
-                if (lane == owner) {
-                    uint64_t run = above + excl;
-                    int e = 0;
-                    for (; e < 8; ++e) {
-                        if (static_cast<double>(run + m8[e]) >= thr) break;
-                        run += m8[e];
-                    }
-                    digit = 255 - 8 * lane - e;
-                    new_above = run;
-                    dcount = hc[digit];
-                }
-                digit = __shfl_sync(0xffffffffu, digit, owner);
-                above = shfl_u64(new_above, owner);
-                dcount = __shfl_sync(0xffffffffu, dcount, owner);
-                prefix = (prefix << 8) | static_cast<uint64_t>(digit);
-                if (dcount == 1 || shift == 0) {
-                    cstar = prefix << shift;
-                    done = true;
-                }
-                __syncwarp();
+            for (int e = 0; e < E; ++e) {
+                const int j = lane + 32 * e;
+                const float sv = j < nb ? srow[j] : 0.f;
+                kv[e] = j < nb ? order_key(sv) : 0u;
+                wv[e] = j < nb ? mass_of(sv, smax) : 0.0;
+                U += wv[e];
             }
+            U = warp_sum(U);
+            const double thr = static_cast<double>(prm.p) * U;
+            // largest score key tau with mass(key >= tau) >= thr
+            uint32_t tau = 0;
+            for (int b = 31; b >= 0; --b) {
+                const uint32_t cand = tau | (1u << b);
+                double m0 = 0.0, m1 = 0.0;
+#pragma unroll
+                for (int e = 0; e < E; e += 2) {
+                    if (kv[e] >= cand) m0 += wv[e];
+                    if (e + 1 < E && kv[e + 1] >= cand) m1 += wv[e + 1];
+                }
+                if (warp_sum(m0 + m1) >= thr) tau = cand;
+            }
+            // blocks sharing the score key tau are taken in ascending index
+            int nt = 0, jt = -1;
+            double above = 0.0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const int j = lane + 32 * e;
+                if (j < nb && kv[e] == tau) {
+                    ++nt;
+                    jt = j;
+                }
+                if (kv[e] > tau) above += wv[e];
+            }
+            for (int o = 16; o > 0; o >>= 1) {
+                nt += __shfl_xor_sync(0xffffffffu, nt, o);
+                jt = max(jt, __shfl_xor_sync(0xffffffffu, jt, o));
+            }
+            uint32_t xs;  // 0xFFFF - index of the last kept block
+            if (nt == 1) {
+                xs = 0xFFFFu - static_cast<uint32_t>(jt);
+            } else {
+                above = warp_sum(above);
+                xs = 0;
+                for (int b = 15; b >= 0; --b) {
+                    const uint32_t cand = xs | (1u << b);
+                    double m = 0.0;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        const int j = lane + 32 * e;
+                        if (j < nb && kv[e] == tau && (0xFFFFu - j) >= cand) m += wv[e];
+                    }
+                    if (above + warp_sum(m) >= thr) xs = cand;
+                }
+            }
+            cstar = (static_cast<uint64_t>(tau) << 16) | xs;
         }
         // emit: bit row + ascending list
         const int ti = i / (prm.Hp * prm.Wp), hi = (i / prm.Wp) % prm.Hp, wi = i % prm.Wp;
@@ -293,16 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          static_cast<uint64_t>(0xFFFFu - j);
                     m = key >= cstar;
                 }
-                m = m || (j == i);
+                m = m || (j == i) || (prm.flags & 2u);
                 if (!m && !(prm.flags & 1u)) {
-                    if (prm.flags & 2u) {
-                        m = true;
-                    } else {
-                        const int tj = j / (prm.Hp * prm.Wp), hj = (j / prm.Wp) % prm.Hp,
-                                  wj = j % prm.Wp;
-                        m = abs(ti - tj) <= prm.wt / 2 && abs(hi - hj) <= prm.wh / 2 &&
-                            abs(wi - wj) <= prm.ww / 2;
-                    }
+                    const int tj = j / (prm.Hp * prm.Wp), hj = (j / prm.Wp) % prm.Hp,
+                              wj = j % prm.Wp;
+                    m = abs(ti - tj) <= prm.wt / 2 && abs(hi - hj) <= prm.wh / 2 &&
+                        abs(wi - wj) <= prm.ww / 2;
                 }
             }
             const unsigned ball = __ballot_sync(0xffffffffu, m);
@@ -358,9 +370,35 @@ __global__ void __launch_bounds__(256) col_lists_kernel(const uint32_t *__restri
 size_t nabla_score_cut_smem(int nb, int D) {
     const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
     const size_t phase1 = sizeof(float) * (static_cast<size_t>(D) * nabla::kRows +
-                                           nabla::kDc * nabla::kCols);
-    const size_t phase2 = 8 * 256 * (sizeof(uint64_t) + sizeof(uint32_t));
-    return sizeof(float) * nabla::kRows * nbp + (phase1 > phase2 ? phase1 : phase2);
+                                           2 * nabla::kDc * nabla::kCols);
+    return sizeof(float) * nabla::kRows * nbp + phase1;
+}
+
+template <int D, int E>
+static cudaError_t launch_score_cut(dim3 grid, size_t smem, const float *qbar,
+                                    const float *kbar_t, nabla::CutParams prm, uint32_t *bits,
+                                    uint16_t *row_idx, int32_t *row_cnt, cudaStream_t stream) {
+    cudaError_t err = cudaFuncSetAttribute(nabla::score_cut_kernel<D, E>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    nabla::score_cut_kernel<D, E><<<grid, nabla::kThreads, smem, stream>>>(qbar, kbar_t, prm, bits,
+                                                                           row_idx, row_cnt);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t dispatch_score_cut(dim3 grid, size_t smem, const float *qbar,
+                                      const float *kbar_t, nabla::CutParams prm, uint32_t *bits,
+                                      uint16_t *row_idx, int32_t *row_cnt, cudaStream_t stream) {
+    const int e = (prm.nb + 31) / 32;
+#define NABLA_SC(EV)                                                                          \
+    if (e <= EV)                                                                              \
+        return launch_score_cut<D, EV>(grid, smem, qbar, kbar_t, prm, bits, row_idx, row_cnt, \
+                                       stream);
+    NABLA_SC(1) NABLA_SC(4) NABLA_SC(16) NABLA_SC(40) NABLA_SC(48) NABLA_SC(64)
+#undef NABLA_SC
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, float p,
@@ -386,19 +424,10 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, f
     CutParams prm{nb, Hp, Wp, wt, wh, ww, flags, p, scale};
     const size_t smem = nabla_score_cut_smem(nb, D);
     const dim3 grid(static_cast<unsigned>(BH * ((nb + kRows - 1) / kRows)));
-    if (D == 128) {
-        err = cudaFuncSetAttribute(score_cut_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem));
-        if (err != cudaSuccess) return err;
-        score_cut_kernel<128><<<grid, kThreads, smem, stream>>>(qbar, kbar_t, prm, bits, row_idx,
-                                                                row_cnt);
-    } else {
-        err = cudaFuncSetAttribute(score_cut_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(smem));
-        if (err != cudaSuccess) return err;
-        score_cut_kernel<64><<<grid, kThreads, smem, stream>>>(qbar, kbar_t, prm, bits, row_idx,
-                                                               row_cnt);
-    }
+    err = D == 128 ? dispatch_score_cut<128>(grid, smem, qbar, kbar_t, prm, bits, row_idx, row_cnt,
+                                             stream)
+                   : dispatch_score_cut<64>(grid, smem, qbar, kbar_t, prm, bits, row_idx, row_cnt,
+                                            stream);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (col_idx) {

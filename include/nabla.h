@@ -155,8 +155,9 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params,
  * -- so cannot provide the scratch nabla_build_mask needs for the pooled
  * means.  Here that scratch is a 32 MiB array compiled into the library: every
  * GPU that loads the library holds those 32 MiB until the process exits.
- *   - Limit: 2 * round_up_256(4 * B*heads * nb * D) <= 32 MiB (e.g. 16 heads of
- *     a 1440-block, D = 128 problem fit; 40 heads of 1200 blocks do not).
+ *   - Limit: round_up_256(4 * B*heads * nb * D) + round_up_256(4 * B*heads * D *
+ *     round_up_4(nb)) <= 32 MiB (e.g. 16 heads of a 1440-block, D = 128
+ *     problem fit; 40 heads of 1200 blocks do not).
  *     Larger shapes return NABLA_ERR_WORKSPACE and enqueue nothing.
  *   - The first call on a device (the current device) looks up the array's
  *     device address with cudaGetSymbolAddress; make that first call before
