@@ -20,6 +20,10 @@ cudaError_t nabla_launch_attn_fwd_mma(int64_t BH, int nb, int D, float scale, co
                                       const void *k, const void *v, const uint16_t *row_idx,
                                       const int32_t *row_cnt, void *o, float *lse,
                                       cudaStream_t stream);
+cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
+                                        const void *q, const void *k, const void *v,
+                                        const uint32_t *bits, void *o, float *lse, int *status,
+                                        int force_timeout, cudaStream_t stream);
 cudaError_t nabla_launch_attn_bwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
                                       const void *k, const void *v, const void *o,
                                       const void *dout, const float *lse, const uint16_t *row_idx,
@@ -67,7 +71,8 @@ int check_params(const nabla_params *p, bool need_window) {
     if (p == nullptr) return NABLA_ERR_NULL;
     if (!(p->p >= 0.f && p->p <= 1.f)) return NABLA_ERR_PARAM;  // also rejects NaN
     if (!(p->scale > 0.f) || !std::isfinite(p->scale)) return NABLA_ERR_PARAM;
-    if ((p->flags & ~(NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS)) != 0) return NABLA_ERR_PARAM;
+    if ((p->flags & ~(NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS | NABLA_DEBUG_TIMEOUT)) != 0)
+        return NABLA_ERR_PARAM;
     if ((p->flags & NABLA_NO_STA) && (p->flags & NABLA_FULL_STA)) return NABLA_ERR_PARAM;
     if (need_window && !(p->flags & (NABLA_NO_STA | NABLA_FULL_STA))) {
         for (int w : {p->sta_t, p->sta_h, p->sta_w})
@@ -186,12 +191,18 @@ int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const n
     if (st != NABLA_OK) return st;
     if ((st = check_params(params, false)) != NABLA_OK) return st;
     if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || mask == nullptr ||
-        mask->row_idx == nullptr || mask->row_cnt == nullptr)
+        mask->bits == nullptr || mask->row_idx == nullptr || mask->row_cnt == nullptr)
         return NABLA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return NABLA_ERR_ALIGN;
     if ((st = check_ws(d, NABLA_OP_ATTN_FWD, workspace, workspace_bytes)) != NABLA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
+    if (d.D == 128) {
+        const int T = shape->T;
+        return cuda_status(nabla_launch_attn_fwd_sm100(
+            d.BH, d.nb, d.Hp, d.Wp, T, params->scale, q, k, v, mask->bits, o, lse,
+            static_cast<int *>(workspace), (params->flags & NABLA_DEBUG_TIMEOUT) ? 1 : 0, s));
+    }
     return cuda_status(nabla_launch_attn_fwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v,
                                                  mask->row_idx, mask->row_cnt, o, lse, s));
 }

@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(HERE, "libnabla.so")
 OK = 0
 ERR_SHAPE, ERR_ALIGN, ERR_PARAM, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_NULL = (
     -1, -2, -3, -4, -5, -6, -7)
-NO_STA, FULL_STA, EMIT_COLS = 1, 2, 4
+NO_STA, FULL_STA, EMIT_COLS, DEBUG_TIMEOUT = 1, 2, 4, 0x100
 OP_BUILD_MASK, OP_ATTN_FWD, OP_ATTN_BWD = 0, 1, 2
 MASK_BITS, MASK_ROW_IDX, MASK_ROW_CNT, MASK_COL_IDX, MASK_COL_CNT = 0, 1, 2, 3, 4
 

@@ -56,6 +56,11 @@ typedef struct CUstream_st *nabla_stream_t; /* == cudaStream_t */
 #define NABLA_NO_STA 1u    /* no STA term: M = adaptive OR diagonal            */
 #define NABLA_FULL_STA 2u  /* STA window covers every block: dense attention   */
 #define NABLA_EMIT_COLS 4u /* also write the column lists needed by the backward */
+/* Test aid, not for production: makes the tensor-core attention forward give
+ * up its first device-side wait at once, so that the timeout path (status
+ * word = NABLA_ERR_TIMEOUT, clean unwind, context still usable) can be
+ * exercised without faulting or hanging the GPU.  Outputs are not written. */
+#define NABLA_DEBUG_TIMEOUT 0x100u
 
 /* Problem shape.  P must be 8. */
 typedef struct {
@@ -177,8 +182,11 @@ int nabla_build_mask_static(const nabla_shape *shape, const nabla_params *params
  *   o_n   = sum over tokens m of blocks j in row i of M of
  *           softmax_m(scale * q_n . k_m) v_m          (bf16 out, fp32 accumulate)
  *   lse_n = log sum_m exp(scale * q_n . k_m)          (float32 [B*heads, N])
- * Needs mask->row_idx and mask->row_cnt.  lse may be NULL when no backward
- * follows.  Workspace: nabla_workspace_size(shape, NABLA_OP_ATTN_FWD). */
+ * Needs mask->bits, mask->row_idx and mask->row_cnt.  lse may be NULL when
+ * no backward follows.  Workspace: nabla_workspace_size(shape,
+ * NABLA_OP_ATTN_FWD).  D = 128 runs on the tcgen05 tensor cores; a device-side
+ * wait that expires (it never should) is reported through nabla_status() and
+ * leaves O and lse unwritten. */
 int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
                    const nabla_bf16 *k, const nabla_bf16 *v, const nabla_mask *mask,
                    nabla_bf16 *o, float *lse, void *workspace, size_t workspace_bytes,

@@ -100,3 +100,23 @@ def test_backward_deterministic():
     assert torch.equal(o, o2)
     for a, b in zip(r1, r2):
         assert torch.equal(a, b)
+
+
+def test_forward_timeout_is_reported_and_the_context_survives():
+    # The test flag makes the forward's first device-side wait give up at once
+    # (a barrier nothing arrives on, with a tiny poll limit): the kernel must
+    # record NABLA_ERR_TIMEOUT, unwind and free its resources; the next call
+    # on the same context must run normally and be correct.
+    w = synth.Workload("odd130", 2, 2, 5, 16, 104, 128, (2, 4, 4), 0.7)
+    c = Case(w)
+    gm = c.gpu_mask()
+    ws = nabla.workspace(c.shape, nabla.OP_ATTN_FWD, "cuda")
+    nabla.attn_fwd(c.shape, c.params(flags=nabla.DEBUG_TIMEOUT), c.gpu["q"], c.gpu["k"],
+                   c.gpu["v"], gm, ws=ws)
+    assert nabla.status(ws) == nabla.ERR_TIMEOUT
+    o, lse = nabla.attn_fwd(c.shape, c.params(), c.gpu["q"], c.gpu["k"], c.gpu["v"], gm, ws=ws)
+    assert nabla.status(ws) == nabla.OK
+    om = c.oracle_mask()
+    q, k, v = (f64(c.cpu[n]) for n in ("q", "k", "v"))
+    oo, _ = oracle.attn_fwd(q, k, v, om["row_idx"], om["row_cnt"], w.scale)
+    assert_close(bf16_to_f64(o).reshape(-1, L, w.D), oo, "O after timeout")
