@@ -24,6 +24,13 @@ cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
                                         const void *q, const void *k, const void *v,
                                         const uint32_t *bits, void *o, float *lse, int *status,
                                         int force_timeout, cudaStream_t stream);
+cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
+                                        const void *q, const void *k, const void *v,
+                                        const void *o, const void *dout, const float *lse,
+                                        const uint16_t *row_idx, const int32_t *row_cnt,
+                                        const uint16_t *col_idx, const int32_t *col_cnt,
+                                        void *dq, void *dk, void *dv, float *dl, float *l2,
+                                        int *status, cudaStream_t stream);
 cudaError_t nabla_launch_attn_bwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
                                       const void *k, const void *v, const void *o,
                                       const void *dout, const float *lse, const uint16_t *row_idx,
@@ -97,8 +104,8 @@ size_t ws_bytes(const Dims &d, int op) {
             return kStatusBytes + mask_scratch_bytes(d);
         case NABLA_OP_ATTN_FWD:
             return kStatusBytes;
-        case NABLA_OP_ATTN_BWD:
-            return kStatusBytes + round256(sizeof(float) * d.BH * d.N);
+        case NABLA_OP_ATTN_BWD:  // D_n and lse_n * log2(e)
+            return kStatusBytes + 2 * round256(sizeof(float) * d.BH * d.N);
         default:
             return 0;
     }
@@ -230,6 +237,14 @@ int nabla_attn_bwd(const nabla_shape *shape, const nabla_params *params, const n
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
     float *dl = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + kStatusBytes);
+    if (d.D == 128) {
+        float *l2 = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(dl) +
+                                              round256(sizeof(float) * d.BH * d.N));
+        return cuda_status(nabla_launch_attn_bwd_sm100(
+            d.BH, d.nb, d.Hp, d.Wp, shape->T, params->scale, q, k, v, o, dout, lse, mask->row_idx,
+            mask->row_cnt, mask->col_idx, mask->col_cnt, dq, dk, dv, dl, l2,
+            static_cast<int *>(workspace), s));
+    }
     return cuda_status(nabla_launch_attn_bwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v, o,
                                                  dout, lse, mask->row_idx, mask->row_cnt,
                                                  mask->col_idx, mask->col_cnt, dq, dk, dv, dl, s));

@@ -1,0 +1,618 @@
+// Block-sparse attention backward on tcgen05 tensor cores, head dim 128.
+//
+// "NABLA: Neighborhood Adaptive Block-Level Attention": training runs through
+// the same block-sparse attention (section 主な貢献, "二段階の加速"), so its
+// gradients are those of attention restricted to the kept 64 x 64 blocks:
+//   D_n = dO_n . O_n,  P = exp(scale q.k - lse),  dS = P (dO.v - D),
+//   dV = P^T dO,  dK = scale dS^T Q,  dQ = scale dS K.
+// Two deterministic kernels (every output tile has one writer, no atomics):
+//
+// dkdv_kernel: one CTA per pair of temporally adjacent KEY blocks (128 key
+//   rows on the M = 128 datapath), walking the union of their mask columns,
+//   one query block (64 queries) per tile:
+//     S^T  = K . Q^T,  dP^T = V . dO^T                 (TMEM, double-buffered)
+//     P^T, dS^T = P^T (dP^T - D)  -> bf16, shared memory (one thread per key)
+//     dV  += P^T . dO,  dK += dS^T . Q                  (TMEM accumulators)
+// dq_kernel: one CTA per query block, walking its mask row two key blocks
+//   (128 keys) per tile:
+//     S^T  = K . Q^T,  dP^T = V . dO^T                 (TMEM, double-buffered)
+//     dS^T                                             (bf16, shared memory)
+//     dQ^T += K^T . dS^T                                (TMEM accumulator)
+// K and V tiles stream through separate TMA rings because K is read twice.
+// All waits are bounded as in the forward.
+#include "sm100.cuh"
+
+namespace nabla {
+namespace bwd100 {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kMaxNbBwd = 2048;
+constexpr uint32_t kHalfTile = 16384;  // 64 rows x 128 features bf16
+constexpr uint32_t kPairTile = 32768;  // 128 rows x 128 features bf16
+
+// ---------------------------------------------------------------------------
+// preprocess: D_n = dO_n . O_n and lse_n * log2(e), 16 threads per row
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restrict__ o,
+                                                  const __nv_bfloat16 *__restrict__ dout,
+                                                  const float *__restrict__ lse,
+                                                  float *__restrict__ dl, float *__restrict__ l2,
+                                                  int64_t rows) {
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
+    const int sub = threadIdx.x & 15;
+    float acc = 0.f;
+    if (row < rows) {
+        const int4 a = *reinterpret_cast<const int4 *>(o + row * kD + sub * 8);
+        const int4 b = *reinterpret_cast<const int4 *>(dout + row * kD + sub * 8);
+        const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
+        const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 u = __bfloat1622float2(x[e]), w = __bfloat1622float2(y[e]);
+            acc = fmaf(u.x, w.x, acc);
+            acc = fmaf(u.y, w.y, acc);
+        }
+    }
+#pragma unroll
+    for (int off = 1; off < 16; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (row < rows && sub == 0) {
+        dl[row] = acc;
+        l2[row] = lse[row] * 1.4426950408889634f;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV
+// ---------------------------------------------------------------------------
+constexpr int kStages = 3;
+constexpr uint32_t kStageBytes = 33792;  // Q 16 KB + dO 16 KB + L2 256 B + D 256 B (+ pad)
+constexpr uint32_t KV_K = 0, KV_V = 32768;
+constexpr uint32_t KV_RING = 65536;
+constexpr uint32_t KV_P = KV_RING + kStages * kStageBytes;  // P^T 16 KB
+constexpr uint32_t KV_DS = KV_P + 16384;                    // dS^T 16 KB
+constexpr uint32_t KV_U = KV_DS + 16384;                    // union list
+constexpr uint32_t KV_UF = KV_U + 2 * (kMaxNbBwd + 8);
+constexpr uint32_t KV_CB = ((KV_UF + kMaxNbBwd + 8 + 15) / 16) * 16;  // column bits [2][64]
+constexpr uint32_t KV_BAR = KV_CB + 2 * 256;
+constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 1;
+constexpr uint32_t KV_INT = KV_BAR + 8 * kKvBars;
+constexpr uint32_t kKvSmem = KV_INT + 16 + 1024;
+
+__global__ void __launch_bounds__(256, 1)
+    dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                const float *__restrict__ l2, const float *__restrict__ dl,
+                const uint16_t *__restrict__ col_idx, const int32_t *__restrict__ col_cnt,
+                __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
+                int *__restrict__ status, int nb, int Hp, int Wp, int T, float c, float scale,
+                uint32_t wait_limit) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+    unsigned char *sm = smem_raw + pad;
+    const uint32_t sb = raw + pad;
+    uint16_t *uList = reinterpret_cast<uint16_t *>(sm + KV_U);
+    uint8_t *uFlag = sm + KV_UF;
+    uint32_t *colBits = reinterpret_cast<uint32_t *>(sm + KV_CB);  // [2][64 words]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + KV_BAR);
+    uint64_t *kv_full = bar, *st_full = bar + 1, *st_empty = bar + 1 + kStages;
+    uint64_t *s_full = bar + 1 + 2 * kStages, *s_empty = s_full + 2, *pd_full = s_empty + 2;
+    uint64_t *pd_empty = pd_full + 1, *done = pd_empty + 1;
+    int *sInt = reinterpret_cast<int *>(sm + KV_INT);
+    volatile int *abort_flag = sInt + 2;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int words = (nb + 31) >> 5;
+    const int HW = Hp * Wp;
+    const int G = ((T + 1) >> 1) * HW;
+    const int64_t bh = blockIdx.x / G;
+    const int g = static_cast<int>(blockIdx.x % G);
+    const int jA = 2 * (g / HW) * HW + g % HW;
+    const int jB = (2 * (g / HW) + 1 < T) ? jA + HW : -1;
+    const int64_t N = static_cast<int64_t>(nb) * kBlk;
+    const int row_base = static_cast<int>(bh * N);
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&st_full[s], 1);
+            mbar_init(&st_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_empty[b], 4);
+        }
+        mbar_init(pd_full, 4);
+        mbar_init(pd_empty, 1);
+        mbar_init(done, 1);
+        sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(reinterpret_cast<uint32_t *>(&sInt[0]), 512);
+        tmem_relinquish();
+    }
+    if (warp == 0) {
+        // column bit masks of jA, jB from the column lists, then their union
+        for (int w = lane; w < 128; w += 32) colBits[w] = 0;
+        __syncwarp();
+        for (int m = 0; m < 2; ++m) {
+            const int j = m ? jB : jA;
+            if (j < 0) continue;
+            const int cnt = col_cnt[bh * nb + j];
+            const uint16_t *lst = col_idx + (bh * nb + j) * static_cast<int64_t>(nb);
+            for (int e = lane; e < cnt; e += 32) {
+                const int i = lst[e];
+                atomicOr(&colBits[m * 64 + (i >> 5)], 1u << (i & 31));
+            }
+        }
+        __syncwarp();
+        const int U = union_bits(colBits, jB >= 0 ? colBits + 64 : nullptr, words, uList, uFlag, lane);
+        if (lane == 0) sInt[1] = U;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = static_cast<uint32_t>(sInt[0]);
+    const int ntiles = *abort_flag ? 0 : sInt[1];  // one query block per tile
+    // TMEM columns: S^T [0,128) (2 x 64), dP^T [128,256) (2 x 64), dV [256,384), dK [384,512)
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tq);
+        prefetch_tmap(&tk);
+        prefetch_tmap(&tv);
+        prefetch_tmap(&tdo);
+        const int ya = row_base + jA * kBlk, yb = row_base + (jB >= 0 ? jB : jA) * kBlk;
+        mbar_expect_tx(kv_full, 2 * kPairTile);
+        for (int dh = 0; dh < 2; ++dh) {
+            tma_load_2d(sb + KV_K + dh * kHalfTile, &tk, kv_full, 64 * dh, ya);
+            tma_load_2d(sb + KV_K + dh * kHalfTile + 8192, &tk, kv_full, 64 * dh, yb);
+            tma_load_2d(sb + KV_V + dh * kHalfTile, &tv, kv_full, 64 * dh, ya);
+            tma_load_2d(sb + KV_V + dh * kHalfTile + 8192, &tv, kv_full, 64 * dh, yb);
+        }
+        int t = 0;
+        for (; t < ntiles; ++t) {
+            const int s = t % kStages;
+            if (!wait_bar(&st_empty[s], ((t / kStages) & 1) ^ 1, abort_flag, status, wait_limit)) break;
+            const uint32_t dst = sb + KV_RING + s * kStageBytes;
+            const int i = uList[t];
+            const int y = row_base + i * kBlk;
+            mbar_expect_tx(&st_full[s], 2 * kHalfTile + 512);
+            tma_load_2d(dst, &tq, &st_full[s], 0, y);
+            tma_load_2d(dst + 8192, &tq, &st_full[s], 64, y);
+            tma_load_2d(dst + 16384, &tdo, &st_full[s], 0, y);
+            tma_load_2d(dst + 24576, &tdo, &st_full[s], 64, y);
+            bulk_load(dst + 32768, l2 + y, 256, &st_full[s]);
+            bulk_load(dst + 33024, dl + y, 256, &st_full[s]);
+        }
+        wait_plain(kv_full, 0, wait_limit);
+        for (int u = t > kStages ? t - kStages : 0; u < t; ++u)
+            wait_plain(&st_full[u % kStages], (u / kStages) & 1, wait_limit);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // K . Q^T, V . dO^T
+            constexpr uint32_t kIdG = idesc_bf16(128, 128, 0, 1);   // P^T . dO, dS^T . Q
+            auto SdP = [&](int t) -> bool {
+                const int s = t % kStages;
+                if (!wait_bar(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
+                    return false;
+                if (!wait_bar(&s_empty[t & 1], ((t >> 1) & 1) ^ 1, abort_flag, status, wait_limit))
+                    return false;
+                tc_fence_after();
+                const uint32_t st = sb + KV_RING + s * kStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                    const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    mma_ss(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
+                           desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
+                    mma_ss(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
+                           desc_sw128(st + 16384 + kb, 16, 1024), kIdS, kk > 0);
+                }
+                mma_commit(&s_full[t & 1]);
+                return true;
+            };
+            auto Grad = [&](int t) -> bool {
+                const int s = t % kStages;
+                if (!wait_bar(pd_full, t & 1, abort_flag, status, wait_limit)) return false;
+                tc_fence_after();
+                const uint32_t st = sb + KV_RING + s * kStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < 64 / 16; ++kk) {
+                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                    mma_ss(tmem + 256, desc_sw128(sb + KV_P + kk * 32, 16, 1024),
+                           desc_sw128(st + 16384 + kk * 2048, 8192, 1024), kIdG, acc);
+                    mma_ss(tmem + 384, desc_sw128(sb + KV_DS + kk * 32, 16, 1024),
+                           desc_sw128(st + kk * 2048, 8192, 1024), kIdG, acc);
+                }
+                mma_commit(pd_empty);
+                mma_commit(&st_empty[s]);
+                return true;
+            };
+            if (ntiles > 0 && wait_bar(kv_full, 0, abort_flag, status, wait_limit)) {
+                bool ok = SdP(0);
+                for (int t = 1; ok && t < ntiles; ++t) ok = SdP(t) && Grad(t - 1);
+                if (ok) Grad(ntiles - 1);
+            }
+            mma_commit(done);
+            wait_plain(done, 0, wait_limit);
+        }
+    } else if (warp >= 4) {
+        const int wq = warp & 3;
+        const int tw = wq * 32 + lane;  // key row 0..127
+        const int kh = tw >> 6;         // key block of the pair
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        bool ok = true;
+        for (int t = 0; t < ntiles; ++t) {
+            ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
+            tc_fence_after();
+            const bool valid = (uFlag[t] >> kh) & 1u;
+            const int s = t % kStages;
+            const float *L = reinterpret_cast<const float *>(sm + KV_RING + s * kStageBytes + 32768);
+            const float *Dv = L + 64;
+            uint32_t pk[32], dk2[32];  // packed bf16 pairs of P^T and dS^T rows
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float sv[32], dp[32];
+                tmem_ld32(tmem + lane_base + (t & 1) * 64 + 32 * half, sv);
+                tmem_ld32(tmem + lane_base + 128 + (t & 1) * 64 + 32 * half, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 l4 = reinterpret_cast<const float4 *>(L)[8 * half + q4];
+                    const float4 d4 = reinterpret_cast<const float4 *>(Dv)[8 * half + q4];
+                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float da[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pv[4], gv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = 4 * q4 + e;
+                        pv[e] = valid ? fast_exp2(fmaf(sv[q], c, -la[e])) : 0.f;
+                        gv[e] = pv[e] * (dp[q] - da[e]);
+                    }
+                    pk[16 * half + 2 * q4] = pack_bf16(pv[0], pv[1]);
+                    pk[16 * half + 2 * q4 + 1] = pack_bf16(pv[2], pv[3]);
+                    dk2[16 * half + 2 * q4] = pack_bf16(gv[0], gv[1]);
+                    dk2[16 * half + 2 * q4 + 1] = pack_bf16(gv[2], gv[3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[t & 1]);
+            if (t > 0) ok = wait_bar(pd_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
+            const uint32_t prow = sb + KV_P + tw * 128, drow = sb + KV_DS + tw * 128;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                const uint32_t off = (cc ^ (tw & 7)) << 4;
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(prow + off),
+                             "r"(pk[4 * cc]), "r"(pk[4 * cc + 1]), "r"(pk[4 * cc + 2]),
+                             "r"(pk[4 * cc + 3])
+                             : "memory");
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(drow + off),
+                             "r"(dk2[4 * cc]), "r"(dk2[4 * cc + 1]), "r"(dk2[4 * cc + 2]),
+                             "r"(dk2[4 * cc + 3])
+                             : "memory");
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pd_full);
+        }
+        if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
+        tc_fence_after();
+        const int jm = kh ? jB : jA;
+        if (jm >= 0 && !*abort_flag) {
+            const int64_t row = bh * N + static_cast<int64_t>(jm) * kBlk + (tw & 63);
+            const bool live = ok && ntiles > 0;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+                __nv_bfloat16 *dst = (which ? dk : dv) + row * kD;
+                const float mul = which ? scale : 1.f;
+#pragma unroll
+                for (int part = 0; part < 4; ++part) {
+                    float v[32];
+                    if (live) {
+                        tmem_ld32(tmem + lane_base + 256 + 128 * which + 32 * part, v);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                        uint4 w;
+                        w.x = pack_bf16(v[8 * e8] * mul, v[8 * e8 + 1] * mul);
+                        w.y = pack_bf16(v[8 * e8 + 2] * mul, v[8 * e8 + 3] * mul);
+                        w.z = pack_bf16(v[8 * e8 + 4] * mul, v[8 * e8 + 5] * mul);
+                        w.w = pack_bf16(v[8 * e8 + 6] * mul, v[8 * e8 + 7] * mul);
+                        *reinterpret_cast<uint4 *>(dst + 32 * part + 8 * e8) = w;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+constexpr int kKSlots = 3, kVSlots = 2;
+constexpr uint32_t DQ_Q = 0, DQ_DO = 16384, DQ_L = 32768, DQ_D = 33024;
+constexpr uint32_t DQ_KR = 34816;                              // 1024-aligned
+constexpr uint32_t DQ_VR = DQ_KR + kKSlots * kPairTile;
+constexpr uint32_t DQ_DS = DQ_VR + kVSlots * kPairTile;        // dS^T 16 KB
+constexpr uint32_t DQ_BAR = DQ_DS + 16384;
+constexpr int kDqBars = 1 + 2 * kKSlots + 2 * kVSlots + 2 + 2 + 1 + 1 + 1;
+constexpr uint32_t DQ_INT = DQ_BAR + 8 * kDqBars;
+constexpr uint32_t kDqSmem = DQ_INT + 16 + 1024;
+
+__global__ void __launch_bounds__(256, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+              const float *__restrict__ l2, const float *__restrict__ dl,
+              const uint16_t *__restrict__ row_idx, const int32_t *__restrict__ row_cnt,
+              __nv_bfloat16 *__restrict__ dq, int *__restrict__ status, int nb, float c,
+              float scale, uint32_t wait_limit) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
+    unsigned char *sm = smem_raw + pad;
+    const uint32_t sb = raw + pad;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + DQ_BAR);
+    uint64_t *q_full = bar, *k_full = bar + 1, *k_empty = k_full + kKSlots;
+    uint64_t *v_full = k_empty + kKSlots, *v_empty = v_full + kVSlots;
+    uint64_t *s_full = v_empty + kVSlots, *s_empty = s_full + 2, *ds_full = s_empty + 2;
+    uint64_t *ds_empty = ds_full + 1, *done = ds_empty + 1;
+    int *sInt = reinterpret_cast<int *>(sm + DQ_INT);
+    volatile int *abort_flag = sInt + 2;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t bh = blockIdx.x / nb;
+    const int i = static_cast<int>(blockIdx.x % nb);
+    const int64_t N = static_cast<int64_t>(nb) * kBlk;
+    const int row_base = static_cast<int>(bh * N);
+    const int cnt = row_cnt[bh * nb + i];
+    const uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kKSlots; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+        }
+        for (int s = 0; s < kVSlots; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_empty[b], 4);
+        }
+        mbar_init(ds_full, 4);
+        mbar_init(ds_empty, 1);
+        mbar_init(done, 1);
+        sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(reinterpret_cast<uint32_t *>(&sInt[0]), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = static_cast<uint32_t>(sInt[0]);
+    const int ntiles = *abort_flag ? 0 : (cnt + 1) >> 1;  // two key blocks per tile
+    // TMEM columns: S^T [0,128) (2 x 64), dP^T [128,256) (2 x 64), dQ^T [256,320)
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tq);
+        prefetch_tmap(&tk);
+        prefetch_tmap(&tv);
+        prefetch_tmap(&tdo);
+        const int y = row_base + i * kBlk;
+        mbar_expect_tx(q_full, 2 * kHalfTile + 512);
+        tma_load_2d(sb + DQ_Q, &tq, q_full, 0, y);
+        tma_load_2d(sb + DQ_Q + 8192, &tq, q_full, 64, y);
+        tma_load_2d(sb + DQ_DO, &tdo, q_full, 0, y);
+        tma_load_2d(sb + DQ_DO + 8192, &tdo, q_full, 64, y);
+        bulk_load(sb + DQ_L, l2 + y, 256, q_full);
+        bulk_load(sb + DQ_D, dl + y, 256, q_full);
+        auto load_pair = [&](const CUtensorMap *tm, uint32_t dst, uint64_t *full, int t) {
+            const int j0 = lst[2 * t];
+            const int j1 = (2 * t + 1 < cnt) ? lst[2 * t + 1] : j0;  // pad with a real block
+            const int y0 = row_base + j0 * kBlk, y1 = row_base + j1 * kBlk;
+            mbar_expect_tx(full, kPairTile);
+            tma_load_2d(dst, tm, full, 0, y0);
+            tma_load_2d(dst + 8192, tm, full, 0, y1);
+            tma_load_2d(dst + 16384, tm, full, 64, y0);
+            tma_load_2d(dst + 24576, tm, full, 64, y1);
+        };
+        int tk_n = 0, tv_n = 0;
+        for (int t = 0; t < ntiles; ++t) {
+            const int ks = t % kKSlots, vs = t % kVSlots;
+            if (!wait_bar(&k_empty[ks], ((t / kKSlots) & 1) ^ 1, abort_flag, status, wait_limit)) break;
+            load_pair(&tk, sb + DQ_KR + ks * kPairTile, &k_full[ks], t);
+            tk_n = t + 1;
+            if (!wait_bar(&v_empty[vs], ((t / kVSlots) & 1) ^ 1, abort_flag, status, wait_limit)) break;
+            load_pair(&tv, sb + DQ_VR + vs * kPairTile, &v_full[vs], t);
+            tv_n = t + 1;
+        }
+        wait_plain(q_full, 0, wait_limit);
+        for (int u = tk_n > kKSlots ? tk_n - kKSlots : 0; u < tk_n; ++u)
+            wait_plain(&k_full[u % kKSlots], (u / kKSlots) & 1, wait_limit);
+        for (int u = tv_n > kVSlots ? tv_n - kVSlots : 0; u < tv_n; ++u)
+            wait_plain(&v_full[u % kVSlots], (u / kVSlots) & 1, wait_limit);
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);   // K . Q^T, V . dO^T
+            constexpr uint32_t kIdQ = idesc_bf16(128, 64, 1, 1);   // K^T . dS^T
+            auto SdP = [&](int t) -> bool {
+                const int ks = t % kKSlots, vs = t % kVSlots;
+                if (!wait_bar(&k_full[ks], (t / kKSlots) & 1, abort_flag, status, wait_limit) ||
+                    !wait_bar(&v_full[vs], (t / kVSlots) & 1, abort_flag, status, wait_limit) ||
+                    !wait_bar(&s_empty[t & 1], ((t >> 1) & 1) ^ 1, abort_flag, status, wait_limit))
+                    return false;
+                tc_fence_after();
+                const uint32_t ka0 = sb + DQ_KR + ks * kPairTile, va0 = sb + DQ_VR + vs * kPairTile;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                    const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    mma_ss(tmem + (t & 1) * 64, desc_sw128(ka0 + ka, 16, 1024),
+                           desc_sw128(sb + DQ_Q + kb, 16, 1024), kIdS, kk > 0);
+                    mma_ss(tmem + 128 + (t & 1) * 64, desc_sw128(va0 + ka, 16, 1024),
+                           desc_sw128(sb + DQ_DO + kb, 16, 1024), kIdS, kk > 0);
+                }
+                mma_commit(&v_empty[vs]);
+                mma_commit(&s_full[t & 1]);
+                return true;
+            };
+            auto Grad = [&](int t) -> bool {
+                const int ks = t % kKSlots;
+                if (!wait_bar(ds_full, t & 1, abort_flag, status, wait_limit)) return false;
+                tc_fence_after();
+                const uint32_t ka0 = sb + DQ_KR + ks * kPairTile;
+#pragma unroll
+                for (int kk = 0; kk < 128 / 16; ++kk)
+                    mma_ss(tmem + 256, desc_sw128(ka0 + kk * 2048, kHalfTile, 1024),
+                           desc_sw128(sb + DQ_DS + kk * 2048, kHalfTile, 1024), kIdQ,
+                           (t > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(ds_empty);
+                mma_commit(&k_empty[ks]);
+                return true;
+            };
+            if (ntiles > 0 && wait_bar(q_full, 0, abort_flag, status, wait_limit)) {
+                bool ok = SdP(0);
+                for (int t = 1; ok && t < ntiles; ++t) ok = SdP(t) && Grad(t - 1);
+                if (ok) Grad(ntiles - 1);
+            }
+            mma_commit(done);
+            wait_plain(done, 0, wait_limit);
+        }
+    } else if (warp >= 4) {
+        const int wq = warp & 3;
+        const int tw = wq * 32 + lane;  // key row 0..127 of the tile
+        const int kh = tw >> 6;
+        const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+        const float *L = reinterpret_cast<const float *>(sm + DQ_L);
+        const float *Dv = reinterpret_cast<const float *>(sm + DQ_D);
+        bool ok = ntiles == 0 || wait_bar(q_full, 0, abort_flag, status, wait_limit);
+        for (int t = 0; t < ntiles; ++t) {
+            ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
+            tc_fence_after();
+            const bool valid = kh == 0 || (2 * t + 1 < cnt);
+            uint32_t gk[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float sv[32], dp[32];
+                tmem_ld32(tmem + lane_base + (t & 1) * 64 + 32 * half, sv);
+                tmem_ld32(tmem + lane_base + 128 + (t & 1) * 64 + 32 * half, dp);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float4 l4 = reinterpret_cast<const float4 *>(L)[8 * half + q4];
+                    const float4 d4 = reinterpret_cast<const float4 *>(Dv)[8 * half + q4];
+                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float da[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float gv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int q = 4 * q4 + e;
+                        const float p = valid ? fast_exp2(fmaf(sv[q], c, -la[e])) : 0.f;
+                        gv[e] = p * (dp[q] - da[e]);
+                    }
+                    gk[16 * half + 2 * q4] = pack_bf16(gv[0], gv[1]);
+                    gk[16 * half + 2 * q4 + 1] = pack_bf16(gv[2], gv[3]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[t & 1]);
+            if (t > 0) ok = wait_bar(ds_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
+            const uint32_t drow = sb + DQ_DS + tw * 128;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc)
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
+                                 drow + ((cc ^ (tw & 7)) << 4)),
+                             "r"(gk[4 * cc]), "r"(gk[4 * cc + 1]), "r"(gk[4 * cc + 2]),
+                             "r"(gk[4 * cc + 3])
+                             : "memory");
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_full);
+        }
+        if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
+        tc_fence_after();
+        if (!*abort_flag) {
+            // thread tw = feature d; dQ^T row d over the 64 queries
+            const int64_t row0 = bh * N + static_cast<int64_t>(i) * kBlk;
+            const bool live = ok && ntiles > 0;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                float v[32];
+                if (live) {
+                    tmem_ld32(tmem + lane_base + 256 + 32 * half, v);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < 32; ++q)
+                    dq[(row0 + 32 * half + q) * kD + tw] = __float2bfloat16_rn(v[q] * scale);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace bwd100
+}  // namespace nabla
+
+cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
+                                        const void *q, const void *k, const void *v,
+                                        const void *o, const void *dout, const float *lse,
+                                        const uint16_t *row_idx, const int32_t *row_cnt,
+                                        const uint16_t *col_idx, const int32_t *col_cnt,
+                                        void *dq, void *dk, void *dv, float *dl, float *l2,
+                                        int *status, cudaStream_t stream) {
+    using namespace nabla::bwd100;
+    const int64_t rows = BH * static_cast<int64_t>(nb) * nabla::kBlk;
+    if (rows >= (1ll << 31) || nb > kMaxNbBwd) return cudaErrorInvalidValue;
+    pre_kernel<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, dl,
+        l2, rows);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    CUtensorMap mq, mk, mv, mdo;
+    if (!nabla_make_tmap_rows128(&mq, q, rows) || !nabla_make_tmap_rows128(&mk, k, rows) ||
+        !nabla_make_tmap_rows128(&mv, v, rows) || !nabla_make_tmap_rows128(&mdo, dout, rows))
+        return cudaErrorInvalidValue;
+    const float c = scale * 1.4426950408889634f;
+    const uint32_t limit = 1u << 20;
+    err = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kKvSmem));
+    if (err != cudaSuccess) return err;
+    const int64_t groups = static_cast<int64_t>((T + 1) / 2) * Hp * Wp;
+    dkdv_kernel<<<static_cast<unsigned>(BH * groups), 256, kKvSmem, stream>>>(
+        mq, mk, mv, mdo, l2, dl, col_idx, col_cnt, static_cast<__nv_bfloat16 *>(dk),
+        static_cast<__nv_bfloat16 *>(dv), status, nb, Hp, Wp, T, c, scale, limit);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kDqSmem));
+    if (err != cudaSuccess) return err;
+    dq_kernel<<<static_cast<unsigned>(BH * nb), 256, kDqSmem, stream>>>(
+        mq, mk, mv, mdo, l2, dl, row_idx, row_cnt, static_cast<__nv_bfloat16 *>(dq), status, nb,
+        c, scale, limit);
+    return cudaGetLastError();
+}

@@ -62,14 +62,6 @@ constexpr int kNumBars = 1 + 2 * kRing + 2 + 2 + 1 + 1 + 1 + 1;
 constexpr uint32_t OFF_INT = OFF_BAR + 8 * kNumBars;              // ints
 constexpr uint32_t kSmemBytes = OFF_INT + 16 + 1024;              // + alignment slack
 
-__device__ __forceinline__ bool wait_plain(uint64_t *bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t n = 0; n < limit; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        __nanosleep(256);
-    }
-    return false;
-}
-
 // Transposed warp reduction of 32 values per lane: afterwards lane l holds
 // the reduction over the warp of column l (in v[0]).
 template <bool MAX>
@@ -150,33 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // union of the two bit rows, ascending, with 2-bit membership
         const uint32_t *ra = bits + (bh * nb + iA) * words;
         const uint32_t *rb = iB >= 0 ? bits + (bh * nb + iB) * words : nullptr;
-        int U = 0;
-        for (int w0 = 0; w0 < words; w0 += 32) {
-            const int w = w0 + lane;
-            uint32_t a = 0, b = 0;
-            if (w < words) {
-                a = ra[w];
-                if (rb) b = rb[w];
-            }
-            uint32_t u = a | b;
-            const int cnt = __popc(u);
-            int incl = cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int t = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += t;
-            }
-            int pos = U + incl - cnt;
-            while (u) {
-                const int bit = __ffs(u) - 1;
-                u &= u - 1;
-                uList[pos] = static_cast<uint16_t>(w * 32 + bit);
-                uFlag[pos] = static_cast<uint8_t>(((a >> bit) & 1u) | (((b >> bit) & 1u) << 1));
-                ++pos;
-            }
-            U += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        __syncwarp();
+        const int U = union_bits(ra, rb, words, uList, uFlag, lane);
         const int ntiles = (U + 1) >> 1;
         for (int t = lane; t < ntiles; t += 32) {
             const int f0 = uFlag[2 * t];
@@ -485,8 +451,10 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+}  // namespace
+
 // [rows, 128] bf16 row-major, boxes of 64 rows x 64 features, 128-byte swizzle
-bool make_map(CUtensorMap *m, const void *base, uint64_t rows) {
+bool nabla_make_tmap_rows128(CUtensorMap *m, const void *base, uint64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t dims[2] = {128, rows};
@@ -498,8 +466,6 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t rows) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
 size_t nabla_fwd_sm100_smem() { return nabla::fwd100::kSmemBytes; }
 
 cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
@@ -510,7 +476,8 @@ cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
     const uint64_t rows = static_cast<uint64_t>(BH) * nb * nabla::kBlk;
     if (rows >= (1ull << 31) || nb > kMaxNbFwd) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, rows) || !make_map(&mk, k, rows) || !make_map(&mv, v, rows))
+    if (!nabla_make_tmap_rows128(&mq, q, rows) || !nabla_make_tmap_rows128(&mk, k, rows) ||
+        !nabla_make_tmap_rows128(&mv, v, rows))
         return cudaErrorInvalidValue;
     cudaError_t err = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            static_cast<int>(kSmemBytes));

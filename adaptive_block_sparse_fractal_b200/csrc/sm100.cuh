@@ -181,5 +181,62 @@ __device__ __forceinline__ void bar_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
 }
 
+// Ascending enumeration of the set bits of (ra | rb) over `words` 32-bit
+// words, by one full warp: list[k] = bit index, flags[k] = bit 0 from ra,
+// bit 1 from rb.  rb may be null.  Returns the number of entries (all lanes).
+__device__ __forceinline__ int union_bits(const uint32_t *ra, const uint32_t *rb, int words,
+                                          uint16_t *list, uint8_t *flags, int lane) {
+    int U = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t a = 0, b = 0;
+        if (w < words) {
+            a = ra[w];
+            if (rb) b = rb[w];
+        }
+        uint32_t u = a | b;
+        const int cnt = __popc(u);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int t = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += t;
+        }
+        int pos = U + incl - cnt;
+        while (u) {
+            const int bit = __ffs(u) - 1;
+            u &= u - 1;
+            list[pos] = static_cast<uint16_t>(w * 32 + bit);
+            flags[pos] = static_cast<uint8_t>(((a >> bit) & 1u) | (((b >> bit) & 1u) << 1));
+            ++pos;
+        }
+        U += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    return U;
+}
+
+// 1-D bulk copy global -> shared (size multiple of 16, both 16-byte aligned).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            dst),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool wait_plain(uint64_t *bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t n = 0; n < limit; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
+        __nanosleep(256);
+    }
+    return false;
+}
+
 }  // namespace sm100
 }  // namespace nabla
+
+// Host: TMA map over a [rows, 128] bf16 row-major tensor, boxes of 64 rows x
+// 64 features, 128-byte swizzle (defined in attn_fwd_sm100.cu).
+bool nabla_make_tmap_rows128(CUtensorMap *m, const void *base, uint64_t rows);

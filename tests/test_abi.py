@@ -52,7 +52,7 @@ def test_sizes(L):
     assert nabla.mask_bytes(s, nabla.MASK_ROW_IDX) == BH * nb * nb * 2
     assert nabla.mask_bytes(s, nabla.MASK_COL_CNT) == BH * nb * 4
     assert nabla.workspace_size(s, nabla.OP_BUILD_MASK) == 256 + 2 * BH * nb * D * 4
-    assert nabla.workspace_size(s, nabla.OP_ATTN_BWD) == 256 + BH * N * 4
+    assert nabla.workspace_size(s, nabla.OP_ATTN_BWD) == 256 + 2 * BH * N * 4
     assert nabla.workspace_size(s, nabla.OP_ATTN_FWD) >= 256
     # invalid shapes size to 0
     for bad in (_shape(P=4), _shape(D=96), _shape(H=50), _shape(T=0), _shape(T=200)):
