@@ -280,7 +280,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld32(saddr, p);
                     tmem_ld32(saddr + 32, p + 32);
                     tmem_wait_ld();
-                    float xm = -INFINITY;
+                    float xm8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) xm8[e] = -INFINITY;
 #pragma unroll
                     for (int q4 = 0; q4 < 16; ++q4) {
                         const float4 m4 = reinterpret_cast<const float4 *>(mrow)[q4];
@@ -288,10 +290,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const float x = fmaf(p[4 * q4 + e], c, -mm[e]);
-                            xm = fmaxf(xm, x);
+                            xm8[(4 * q4 + e) & 7] = fmaxf(xm8[(4 * q4 + e) & 7], x);
                             p[4 * q4 + e] = valid ? fast_exp2(x) : 0.f;
                         }
                     }
+                    const float xm = fmaxf(fmaxf(fmaxf(xm8[0], xm8[1]), fmaxf(xm8[2], xm8[3])),
+                                           fmaxf(fmaxf(xm8[4], xm8[5]), fmaxf(xm8[6], xm8[7])));
                     need = bar_or(barid, 128, valid && xm > kRescaleAt);
                 }
                 if (need) {

@@ -50,7 +50,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
             atomicExch(status, kDevTimeout);
             return false;
         }
-        if (n > 32) __nanosleep(128);
+        if (n > 4096) __nanosleep(64);  // long waits only: short ones stay on the fast path
     }
     return true;
 }

@@ -45,7 +45,22 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=("train", "long"),
+                    help="train: 720p-like training step (the benchmark); long: 92,160-token clip")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run fewer heads (profiling captures only; not a benchmark result)")
     return ap.parse_args()
+
+
+def workload_of(args):
+    import dataclasses
+    from adaptive_block_sparse_fractal_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.workload == "long":
+        w = dataclasses.replace(w, backward=True)
+    if args.heads is not None:
+        w = dataclasses.replace(w, heads=args.heads)
+    return w
 
 
 def peaks():
@@ -59,9 +74,10 @@ def peaks():
 
 def workload_config(w):
     return {
-        "workload": "train-720p: B=%d heads=%d T*H*W=%dx%dx%d (%d tokens, %d blocks of 64) D=%d "
+        "workload": "%s: B=%d heads=%d T*H*W=%dx%dx%d (%d tokens, %d blocks of 64) D=%d "
                     "p=%.2f STA %dx%dx%d; flatten + mask + fwd + bwd + unflatten"
-                    % (w.B, w.heads, w.T, w.H, w.W, w.N, w.nb, w.D, w.p, *w.window),
+                    % ("train-720p" if w.name == "train" else w.name, w.B, w.heads, w.T, w.H, w.W,
+                       w.N, w.nb, w.D, w.p, *w.window),
         "global_batch": w.B,
         "seq_len": w.N,
         "heads": w.heads,
@@ -174,8 +190,7 @@ def run_reference(args):
     rank, world, _ = dist_init(args.gpus)
     if rank != 0:
         return 0
-    from adaptive_block_sparse_fractal_b200 import synth
-    w = synth.WORKLOADS[WORKLOAD]
+    w = workload_of(args)
     times, flops = [], []
     for s in range(args.warmup + args.steps):
         t0 = time.perf_counter()
@@ -211,7 +226,7 @@ def run_nabla(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     nabla.lib()
-    w = synth.WORKLOADS[WORKLOAD]
+    w = workload_of(args)
     shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
     prm = nabla.params_of(w.p, w.window, D=w.D, flags=nabla.EMIT_COLS)
 
