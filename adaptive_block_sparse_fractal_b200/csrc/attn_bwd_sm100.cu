@@ -301,10 +301,13 @@ __global__ void __launch_bounds__(256, 1)
         }
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
+        // warp-uniform flags around the collective TMEM loads
+        const bool aborted = __any_sync(0xffffffffu, *abort_flag != 0);
+        const bool all_ok = __all_sync(0xffffffffu, ok);
         const int jm = kh ? jB : jA;
-        if (jm >= 0 && !*abort_flag) {
+        if (jm >= 0 && !aborted) {
             const int64_t row = bh * N + static_cast<int64_t>(jm) * kBlk + (tw & 63);
-            const bool live = ok && ntiles > 0;
+            const bool live = all_ok && ntiles > 0;
 #pragma unroll
             for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
                 __nv_bfloat16 *dst = (which ? dk : dv) + row * kD;
@@ -549,10 +552,13 @@ __global__ void __launch_bounds__(256, 1)
         }
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
-        if (!*abort_flag) {
+        // warp-uniform flags around the collective TMEM loads
+        const bool aborted = __any_sync(0xffffffffu, *abort_flag != 0);
+        const bool all_ok = __all_sync(0xffffffffu, ok);
+        if (!aborted) {
             // thread tw = feature d; dQ^T row d over the 64 queries
             const int64_t row0 = bh * N + static_cast<int64_t>(i) * kBlk;
-            const bool live = ok && ntiles > 0;
+            const bool live = all_ok && ntiles > 0;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 float v[32];
@@ -598,7 +604,7 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
         !nabla_make_tmap_rows128(&mv, v, rows) || !nabla_make_tmap_rows128(&mdo, dout, rows))
         return cudaErrorInvalidValue;
     const float c = scale * 1.4426950408889634f;
-    const uint32_t limit = 1u << 20;
+    const uint32_t limit = 1000000000u;  // 1 s per wait
     err = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kKvSmem));
     if (err != cudaSuccess) return err;

@@ -36,23 +36,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+
 // Bounded wait for the phase of parity `parity` to complete.  Gives up when
-// another thread of the CTA has aborted (abort flag set) or after `limit`
-// unsuccessful polls, in which case it sets the abort flag and the status
+// another thread of the CTA has aborted (abort flag set) or after `limit_ns`
+// nanoseconds of waiting, in which case it sets the abort flag and the status
 // word.  Returns false when it gave up.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                         int *status, uint32_t limit) {
-    uint32_t n = 0;
-    while (!mbar_try_wait(bar, parity)) {
+                                         int *status, uint32_t limit_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t n = 0;; ++n) {
+        if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (++n > limit) {
-            *abort = 1;
-            atomicExch(status, kDevTimeout);
-            return false;
+        if ((n & 63) == 63) {
+            if (global_ns() - t0 > limit_ns) {
+                *abort = 1;
+                atomicExch(status, kDevTimeout);
+                return false;
+            }
+            if (n > 4096) __nanosleep(64);  // long waits only
         }
-        if (n > 4096) __nanosleep(64);  // long waits only: short ones stay on the fast path
     }
-    return true;
 }
 
 // ---- TMA --------------------------------------------------------------------
@@ -93,6 +102,15 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16; A is M x K, K-major, 16-bit
+// elements packed two per 32-bit column (a K = 16 step spans 8 columns).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 // Arrive on `bar` once all previously issued tcgen05 ops of this thread are done.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
@@ -226,12 +244,14 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
-__device__ __forceinline__ bool wait_plain(uint64_t *bar, uint32_t parity, uint32_t limit) {
-    for (uint32_t n = 0; n < limit; ++n) {
-        if (mbar_try_wait(bar, parity)) return true;
-        __nanosleep(256);
+// Bounded wait that ignores the abort flag (used to drain in-flight work).
+__device__ __forceinline__ bool wait_plain(uint64_t *bar, uint32_t parity, uint32_t limit_ns) {
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (global_ns() - t0 > limit_ns) return false;
+        __nanosleep(128);
     }
-    return false;
+    return true;
 }
 
 }  // namespace sm100

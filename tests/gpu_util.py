@@ -19,12 +19,14 @@ FRAGILE_UNITS = 64.0  # a cut decided within 64 units of 2^-40 mass
 class Case:
     """A workload with inputs on both sides."""
 
-    def __init__(self, w, seed0=0, p=None, flags=0, backward=None, device="cuda"):
+    def __init__(self, w, seed0=0, p=None, flags=0, backward=None, device="cuda", mutate=None):
         self.w = w
         self.p = w.p if p is None else p
         self.flags = flags
         self.backward = w.backward if backward is None else backward
         inp = synth.make_inputs(w, seed0, with_dout=self.backward)
+        if mutate is not None:  # a test's deliberate change to the inputs, applied to both sides
+            mutate(inp)
         self.shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
         self.cpu = {}
         self.gpu = {}
