@@ -13,12 +13,11 @@
 //     S^T  = K . Q^T,  dP^T = V . dO^T                 (TMEM, double-buffered)
 //     P^T, dS^T = P^T (dP^T - D)  -> bf16, shared memory (one thread per key)
 //     dV  += P^T . dO,  dK += dS^T . Q                  (TMEM accumulators)
-// dq_kernel: one CTA per query block, walking its mask row two key blocks
-//   (128 keys) per tile:
-//     S^T  = K . Q^T,  dP^T = V . dO^T                 (TMEM, double-buffered)
-//     dS^T                                             (bf16, shared memory)
-//     dQ^T += K^T . dS^T                                (TMEM accumulator)
-// K and V tiles stream through separate TMA rings because K is read twice.
+// dq_kernel: one CTA per pair of temporally adjacent QUERY blocks (128 query
+//   rows), walking the union of their mask rows, one key block per tile:
+//     S = Q . K^T,  dP = dO . V^T     (Q, dO resident in TMEM as A operands)
+//     dS = P (dP - D)                  (bf16, written over S in TMEM)
+//     dQ += dS . K                     (TMEM accumulator)
 // All waits are bounded as in the forward.
 #include "sm100.cuh"
 
@@ -344,60 +343,74 @@ __global__ void __launch_bounds__(256, 1)
 // ---------------------------------------------------------------------------
 // dQ
 // ---------------------------------------------------------------------------
-constexpr int kKSlots = 3, kVSlots = 2;
-constexpr uint32_t DQ_Q = 0, DQ_DO = 16384, DQ_L = 32768, DQ_D = 33024;
-constexpr uint32_t DQ_KR = 34816;                              // 1024-aligned
-constexpr uint32_t DQ_VR = DQ_KR + kKSlots * kPairTile;
-constexpr uint32_t DQ_DS = DQ_VR + kVSlots * kPairTile;        // dS^T 16 KB
-constexpr uint32_t DQ_BAR = DQ_DS + 16384;
-constexpr int kDqBars = 1 + 2 * kKSlots + 2 * kVSlots + 2 + 2 + 1 + 1 + 1;
+// One CTA per pair of temporally adjacent QUERY blocks (128 query rows on the
+// M = 128 datapath, the same pairing as the forward), walking the union of
+// their mask rows one key block (64 keys) per tile:
+//   S  = Q . K^T,  dP = dO . V^T    (Q, dO are TMEM A operands; S, dP double-
+//                                    buffered in TMEM)
+//   dS = P (dP - D)  -> bf16, written over S in TMEM (one thread per query)
+//   dQ += dS . K                     (dS the TMEM A operand, K from shared
+//                                    memory, MN-major; accumulator in TMEM)
+// Queries of the pair whose own row does not keep a key block get dS = 0.
+// TMEM columns: buffer b in [128 b, 128 b + 128) holds S (64) then dP (64);
+// dQ [256, 384), Q [384, 448), dO [448, 512).
+constexpr int kDqThreads = 192;
+constexpr int kDqRing = 6;
+constexpr uint32_t kDqSlot = 32768;  // K block 16 KB + V block 16 KB
+constexpr uint32_t kColDQ = 256, kColQ = 384, kColDO = 448;
+constexpr uint32_t DQ_RING = 0;
+constexpr uint32_t DQ_RB = DQ_RING + kDqRing * kDqSlot;   // row bits [2][64]
+constexpr uint32_t DQ_U = DQ_RB + 2 * 256;                // union list u16
+constexpr uint32_t DQ_UF = DQ_U + 2 * (kMaxNbBwd + 8);    // membership per entry
+constexpr uint32_t DQ_BAR = ((DQ_UF + kMaxNbBwd + 8 + 7) / 8) * 8;
+constexpr int kDqBars = 2 * kDqRing + 2 + 2 + 1 + 1;
 constexpr uint32_t DQ_INT = DQ_BAR + 8 * kDqBars;
 constexpr uint32_t kDqSmem = DQ_INT + 16 + 1024;
 
-__global__ void __launch_bounds__(256, 1)
-    dq_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-              const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+__global__ void __launch_bounds__(kDqThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+              const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ dout,
               const float *__restrict__ l2, const float *__restrict__ dl,
               const uint16_t *__restrict__ row_idx, const int32_t *__restrict__ row_cnt,
-              __nv_bfloat16 *__restrict__ dq, int *__restrict__ status, int nb, float c,
-              float scale, uint32_t wait_limit) {
+              __nv_bfloat16 *__restrict__ dq, int *__restrict__ status, int nb, int Hp, int Wp,
+              int T, float c, float scale, uint32_t wait_limit) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
     unsigned char *sm = smem_raw + pad;
-    const uint32_t sb = raw + pad;
+    const uint32_t sRing = raw + pad + DQ_RING;
+    uint32_t *rowBits = reinterpret_cast<uint32_t *>(sm + DQ_RB);  // [2][64 words]
+    uint16_t *uList = reinterpret_cast<uint16_t *>(sm + DQ_U);
+    uint8_t *uFlag = sm + DQ_UF;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + DQ_BAR);
-    uint64_t *q_full = bar, *k_full = bar + 1, *k_empty = k_full + kKSlots;
-    uint64_t *v_full = k_empty + kKSlots, *v_empty = v_full + kVSlots;
-    uint64_t *s_full = v_empty + kVSlots, *s_empty = s_full + 2, *ds_full = s_empty + 2;
-    uint64_t *ds_empty = ds_full + 1, *done = ds_empty + 1;
-    int *sInt = reinterpret_cast<int *>(sm + DQ_INT);
+    uint64_t *kv_full = bar, *kv_empty = bar + kDqRing, *s_full = bar + 2 * kDqRing;
+    // ds_full[t & 1]: the four dS warps wrote dS(t) (two barriers, so a warp
+    // already on tile t+1 cannot complete tile t's phase for the others)
+    uint64_t *ds_full = s_full + 2, *q_ready = ds_full + 2, *done = q_ready + 1;
+    int *sInt = reinterpret_cast<int *>(sm + DQ_INT);  // [0] tmem base [1] tiles [2] abort
     volatile int *abort_flag = sInt + 2;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t bh = blockIdx.x / nb;
-    const int i = static_cast<int>(blockIdx.x % nb);
+    const int words = (nb + 31) >> 5;
+    const int HW = Hp * Wp;
+    const int G = ((T + 1) >> 1) * HW;
+    const int64_t bh = blockIdx.x / G;
+    const int g = static_cast<int>(blockIdx.x % G);
+    const int iA = 2 * (g / HW) * HW + g % HW;
+    const int iB = (2 * (g / HW) + 1 < T) ? iA + HW : -1;
     const int64_t N = static_cast<int64_t>(nb) * kBlk;
     const int row_base = static_cast<int>(bh * N);
-    const int cnt = row_cnt[bh * nb + i];
-    const uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
 
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        for (int s = 0; s < kKSlots; ++s) {
-            mbar_init(&k_full[s], 1);
-            mbar_init(&k_empty[s], 1);
-        }
-        for (int s = 0; s < kVSlots; ++s) {
-            mbar_init(&v_full[s], 1);
-            mbar_init(&v_empty[s], 1);
+        for (int r = 0; r < kDqRing; ++r) {
+            mbar_init(&kv_full[r], 1);
+            mbar_init(&kv_empty[r], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 4);
+            mbar_init(&ds_full[b], 4);
         }
-        mbar_init(ds_full, 4);
-        mbar_init(ds_empty, 1);
+        mbar_init(q_ready, 4);
         mbar_init(done, 1);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
@@ -406,172 +419,189 @@ __global__ void __launch_bounds__(256, 1)
         tmem_alloc(reinterpret_cast<uint32_t *>(&sInt[0]), 512);
         tmem_relinquish();
     }
+    if (warp == 0) {
+        // bit rows of iA, iB from the row lists, then their union
+        for (int w = lane; w < 128; w += 32) rowBits[w] = 0;
+        __syncwarp();
+        for (int m = 0; m < 2; ++m) {
+            const int i = m ? iB : iA;
+            if (i < 0) continue;
+            const int cnt = row_cnt[bh * nb + i];
+            const uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
+            for (int e = lane; e < cnt; e += 32) {
+                const int j = lst[e];
+                atomicOr(&rowBits[m * 64 + (j >> 5)], 1u << (j & 31));
+            }
+        }
+        __syncwarp();
+        const int U = union_bits(rowBits, iB >= 0 ? rowBits + 64 : nullptr, words, uList, uFlag,
+                                 lane);
+        if (lane == 0) sInt[1] = U;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = static_cast<uint32_t>(sInt[0]);
-    const int ntiles = *abort_flag ? 0 : (cnt + 1) >> 1;  // two key blocks per tile
-    // TMEM columns: S^T [0,128) (2 x 64), dP^T [128,256) (2 x 64), dQ^T [256,320)
+    const int ntiles = *abort_flag ? 0 : sInt[1];  // one key block per tile
 
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tq);
+        // ---------------- producer: K and V blocks through the ring ----------------
         prefetch_tmap(&tk);
         prefetch_tmap(&tv);
-        prefetch_tmap(&tdo);
-        const int y = row_base + i * kBlk;
-        mbar_expect_tx(q_full, 2 * kHalfTile + 512);
-        tma_load_2d(sb + DQ_Q, &tq, q_full, 0, y);
-        tma_load_2d(sb + DQ_Q + 8192, &tq, q_full, 64, y);
-        tma_load_2d(sb + DQ_DO, &tdo, q_full, 0, y);
-        tma_load_2d(sb + DQ_DO + 8192, &tdo, q_full, 64, y);
-        bulk_load(sb + DQ_L, l2 + y, 256, q_full);
-        bulk_load(sb + DQ_D, dl + y, 256, q_full);
-        auto load_pair = [&](const CUtensorMap *tm, uint32_t dst, uint64_t *full, int t) {
-            const int j0 = lst[2 * t];
-            const int j1 = (2 * t + 1 < cnt) ? lst[2 * t + 1] : j0;  // pad with a real block
-            const int y0 = row_base + j0 * kBlk, y1 = row_base + j1 * kBlk;
-            mbar_expect_tx(full, kPairTile);
-            tma_load_2d(dst, tm, full, 0, y0);
-            tma_load_2d(dst + 8192, tm, full, 0, y1);
-            tma_load_2d(dst + 16384, tm, full, 64, y0);
-            tma_load_2d(dst + 24576, tm, full, 64, y1);
-        };
-        int tk_n = 0, tv_n = 0;
-        for (int t = 0; t < ntiles; ++t) {
-            const int ks = t % kKSlots, vs = t % kVSlots;
-            if (!wait_bar(&k_empty[ks], ((t / kKSlots) & 1) ^ 1, abort_flag, status, wait_limit)) break;
-            load_pair(&tk, sb + DQ_KR + ks * kPairTile, &k_full[ks], t);
-            tk_n = t + 1;
-            if (!wait_bar(&v_empty[vs], ((t / kVSlots) & 1) ^ 1, abort_flag, status, wait_limit)) break;
-            load_pair(&tv, sb + DQ_VR + vs * kPairTile, &v_full[vs], t);
-            tv_n = t + 1;
+        int t = 0;
+        for (; t < ntiles; ++t) {
+            const int slot = t % kDqRing;
+            if (!wait_bar(&kv_empty[slot], ((t / kDqRing) & 1) ^ 1, abort_flag, status, wait_limit))
+                break;
+            const uint32_t dst = sRing + slot * kDqSlot;
+            const int y = row_base + uList[t] * kBlk;
+            mbar_expect_tx(&kv_full[slot], kDqSlot);
+            tma_load_2d(dst, &tk, &kv_full[slot], 0, y);
+            tma_load_2d(dst + 8192, &tk, &kv_full[slot], 64, y);
+            tma_load_2d(dst + 16384, &tv, &kv_full[slot], 0, y);
+            tma_load_2d(dst + 24576, &tv, &kv_full[slot], 64, y);
         }
-        wait_plain(q_full, 0, wait_limit);
-        for (int u = tk_n > kKSlots ? tk_n - kKSlots : 0; u < tk_n; ++u)
-            wait_plain(&k_full[u % kKSlots], (u / kKSlots) & 1, wait_limit);
-        for (int u = tv_n > kVSlots ? tv_n - kVSlots : 0; u < tv_n; ++u)
-            wait_plain(&v_full[u % kVSlots], (u / kVSlots) & 1, wait_limit);
+        // drain: never leave with a copy in flight
+        for (int u = t > kDqRing ? t - kDqRing : 0; u < t; ++u)
+            wait_plain(&kv_full[u % kDqRing], (u / kDqRing) & 1, wait_limit);
     } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);   // K . Q^T, V . dO^T
-            constexpr uint32_t kIdQ = idesc_bf16(128, 64, 1, 1);   // K^T . dS^T
+            constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // Q . K^T, dO . V^T
+            constexpr uint32_t kIdQ = idesc_bf16(128, 128, 0, 1);   // dS . K (K MN-major)
             auto SdP = [&](int t) -> bool {
-                const int ks = t % kKSlots, vs = t % kVSlots;
-                if (!wait_bar(&k_full[ks], (t / kKSlots) & 1, abort_flag, status, wait_limit) ||
-                    !wait_bar(&v_full[vs], (t / kVSlots) & 1, abort_flag, status, wait_limit) ||
-                    !wait_bar(&s_empty[t & 1], ((t >> 1) & 1) ^ 1, abort_flag, status, wait_limit))
+                const int slot = t % kDqRing;
+                if (!wait_bar(&kv_full[slot], (t / kDqRing) & 1, abort_flag, status, wait_limit))
                     return false;
                 tc_fence_after();
-                const uint32_t ka0 = sb + DQ_KR + ks * kPairTile, va0 = sb + DQ_VR + vs * kPairTile;
+                const uint32_t b0 = sRing + slot * kDqSlot;
+                const uint32_t d = tmem + (t & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                    const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_ss(tmem + (t & 1) * 64, desc_sw128(ka0 + ka, 16, 1024),
-                           desc_sw128(sb + DQ_Q + kb, 16, 1024), kIdS, kk > 0);
-                    mma_ss(tmem + 128 + (t & 1) * 64, desc_sw128(va0 + ka, 16, 1024),
-                           desc_sw128(sb + DQ_DO + kb, 16, 1024), kIdS, kk > 0);
+                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    mma_ts(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
+                    mma_ts(d + 64, tmem + kColDO + 8 * kk, desc_sw128(b0 + 16384 + off, 16, 1024),
+                           kIdS, kk > 0);
                 }
-                mma_commit(&v_empty[vs]);
                 mma_commit(&s_full[t & 1]);
                 return true;
             };
             auto Grad = [&](int t) -> bool {
-                const int ks = t % kKSlots;
-                if (!wait_bar(ds_full, t & 1, abort_flag, status, wait_limit)) return false;
+                const int slot = t % kDqRing;
+                if (!wait_bar(&ds_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit))
+                    return false;
                 tc_fence_after();
-                const uint32_t ka0 = sb + DQ_KR + ks * kPairTile;
+                const uint32_t b0 = sRing + slot * kDqSlot;
 #pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk)
-                    mma_ss(tmem + 256, desc_sw128(ka0 + kk * 2048, kHalfTile, 1024),
-                           desc_sw128(sb + DQ_DS + kk * 2048, kHalfTile, 1024), kIdQ,
-                           (t > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(ds_empty);
-                mma_commit(&k_empty[ks]);
+                for (int kk = 0; kk < 64 / 16; ++kk)
+                    mma_ts(tmem + kColDQ, tmem + (t & 1) * 128 + 8 * kk,
+                           desc_sw128(b0 + kk * 2048, 8192, 1024), kIdQ, (t > 0 || kk > 0));
+                mma_commit(&kv_empty[slot]);
                 return true;
             };
-            if (ntiles > 0 && wait_bar(q_full, 0, abort_flag, status, wait_limit)) {
+            if (ntiles > 0 && wait_bar(q_ready, 0, abort_flag, status, wait_limit)) {
                 bool ok = SdP(0);
-                for (int t = 1; ok && t < ntiles; ++t) ok = SdP(t) && Grad(t - 1);
-                if (ok) Grad(ntiles - 1);
+                for (int t = 0; ok && t < ntiles; ++t) {
+                    if (t + 1 < ntiles) ok = SdP(t + 1);
+                    ok = ok && Grad(t);
+                }
             }
-            mma_commit(done);
+            mma_commit(done);  // completes once every MMA issued above has finished
             wait_plain(done, 0, wait_limit);
         }
-    } else if (warp >= 4) {
-        const int wq = warp & 3;
-        const int tw = wq * 32 + lane;  // key row 0..127 of the tile
-        const int kh = tw >> 6;
+    } else if (warp >= 2) {
+        // ---------------- dS warpgroup: one thread per query row ----------------
+        const int wq = warp & 3;                    // TMEM lane quarter of this warp
+        const int r = wq * 32 + lane;               // query row of the pair, 0..127
+        const int h = r >> 6;                       // 0 -> block iA, 1 -> block iB
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-        const float *L = reinterpret_cast<const float *>(sm + DQ_L);
-        const float *Dv = reinterpret_cast<const float *>(sm + DQ_D);
-        bool ok = ntiles == 0 || wait_bar(q_full, 0, abort_flag, status, wait_limit);
+        const int ib = h ? (iB >= 0 ? iB : iA) : iA;
+        const int64_t grow = bh * N + static_cast<int64_t>(ib) * kBlk + (r & 63);
+        const float Lr = l2[grow], Dr = dl[grow];
+        // Q and dO rows -> TMEM (the A operands of S and dP)
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const uint4 *src = reinterpret_cast<const uint4 *>((which ? dout : q) + grow * kD);
+            const uint32_t col = which ? kColDO : kColQ;
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t v32[32];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const uint4 v = __ldg(src + 8 * half + e);
+                    v32[4 * e] = v.x;
+                    v32[4 * e + 1] = v.y;
+                    v32[4 * e + 2] = v.z;
+                    v32[4 * e + 3] = v.w;
+                }
+                tmem_st32(tmem + lane_base + col + 32 * half, reinterpret_cast<float *>(v32));
+            }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(q_ready);
+
+        bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
-            const bool valid = kh == 0 || (2 * t + 1 < cnt);
+            const bool valid = (uFlag[t] >> h) & 1u;  // uniform per warp
+            const uint32_t scol = tmem + lane_base + (t & 1) * 128;
             uint32_t gk[32];
+            if (valid) {
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float sv[32], dp[32];
-                tmem_ld32(tmem + lane_base + (t & 1) * 64 + 32 * half, sv);
-                tmem_ld32(tmem + lane_base + 128 + (t & 1) * 64 + 32 * half, dp);
-                tmem_wait_ld();
+                for (int half = 0; half < 2; ++half) {
+                    float sv[32], dp[32];
+                    tmem_ld32(scol + 32 * half, sv);
+                    tmem_ld32(scol + 64 + 32 * half, dp);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 l4 = reinterpret_cast<const float4 *>(L)[8 * half + q4];
-                    const float4 d4 = reinterpret_cast<const float4 *>(Dv)[8 * half + q4];
-                    const float la[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float da[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float gv[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int q = 4 * q4 + e;
-                        const float p = valid ? fast_exp2(fmaf(sv[q], c, -la[e])) : 0.f;
-                        gv[e] = p * (dp[q] - da[e]);
+                    for (int e = 0; e < 32; e += 2) {
+                        const float p0 = fast_exp2(fmaf(sv[e], c, -Lr));
+                        const float p1 = fast_exp2(fmaf(sv[e + 1], c, -Lr));
+                        gk[16 * half + (e >> 1)] = pack_bf16(p0 * (dp[e] - Dr), p1 * (dp[e + 1] - Dr));
                     }
-                    gk[16 * half + 2 * q4] = pack_bf16(gv[0], gv[1]);
-                    gk[16 * half + 2 * q4 + 1] = pack_bf16(gv[2], gv[3]);
                 }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) gk[e] = 0u;
             }
+            // bf16 dS over the first 32 columns of this S buffer
+            tmem_st32(scol, reinterpret_cast<float *>(gk));
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[t & 1]);
-            if (t > 0) ok = wait_bar(ds_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
-            const uint32_t drow = sb + DQ_DS + tw * 128;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc)
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(
-                                 drow + ((cc ^ (tw & 7)) << 4)),
-                             "r"(gk[4 * cc]), "r"(gk[4 * cc + 1]), "r"(gk[4 * cc + 2]),
-                             "r"(gk[4 * cc + 3])
-                             : "memory");
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(ds_full);
+            if (lane == 0) mbar_arrive(&ds_full[t & 1]);
         }
+        // ---------------- epilogue ----------------
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
         // warp-uniform flags around the collective TMEM loads
         const bool aborted = __any_sync(0xffffffffu, *abort_flag != 0);
-        const bool all_ok = __all_sync(0xffffffffu, ok);
-        if (!aborted) {
-            // thread tw = feature d; dQ^T row d over the 64 queries
-            const int64_t row0 = bh * N + static_cast<int64_t>(i) * kBlk;
-            const bool live = all_ok && ntiles > 0;
+        const bool have = (h == 0 || iB >= 0) && !aborted;
+        const bool live = have && ntiles > 0 && __all_sync(0xffffffffu, ok);
+        if (have) {
+            __nv_bfloat16 *dst = dq + grow * kD;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int part = 0; part < 4; ++part) {
                 float v[32];
                 if (live) {
-                    tmem_ld32(tmem + lane_base + 256 + 32 * half, v);
+                    tmem_ld32(tmem + lane_base + kColDQ + 32 * part, v);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) v[e] = 0.f;
                 }
 #pragma unroll
-                for (int q = 0; q < 32; ++q)
-                    dq[(row0 + 32 * half + q) * kD + tw] = __float2bfloat16_rn(v[q] * scale);
+                for (int e8 = 0; e8 < 4; ++e8) {
+                    uint4 w;
+                    w.x = pack_bf16(v[8 * e8] * scale, v[8 * e8 + 1] * scale);
+                    w.y = pack_bf16(v[8 * e8 + 2] * scale, v[8 * e8 + 3] * scale);
+                    w.z = pack_bf16(v[8 * e8 + 4] * scale, v[8 * e8 + 5] * scale);
+                    w.w = pack_bf16(v[8 * e8 + 6] * scale, v[8 * e8 + 7] * scale);
+                    *reinterpret_cast<uint4 *>(dst + 32 * part + 8 * e8) = w;
+                }
             }
         }
     }
@@ -580,7 +610,6 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
-
 }  // namespace bwd100
 }  // namespace nabla
 
@@ -617,8 +646,9 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
     err = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kDqSmem));
     if (err != cudaSuccess) return err;
-    dq_kernel<<<static_cast<unsigned>(BH * nb), 256, kDqSmem, stream>>>(
-        mq, mk, mv, mdo, l2, dl, row_idx, row_cnt, static_cast<__nv_bfloat16 *>(dq), status, nb,
-        c, scale, limit);
+    dq_kernel<<<static_cast<unsigned>(BH * groups), kDqThreads, kDqSmem, stream>>>(
+        mk, mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(dout),
+        l2, dl, row_idx, row_cnt, static_cast<__nv_bfloat16 *>(dq), status, nb, Hp, Wp, T, c,
+        scale, limit);
     return cudaGetLastError();
 }
