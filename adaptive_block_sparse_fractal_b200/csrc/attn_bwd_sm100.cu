@@ -190,54 +190,54 @@ __global__ void __launch_bounds__(256, 1)
         for (int u = t > kStages ? t - kStages : 0; u < t; ++u)
             wait_plain(&st_full[u % kStages], (u / kStages) & 1, wait_limit);
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // K . Q^T, V . dO^T
-            constexpr uint32_t kIdG = idesc_bf16(128, 128, 0, 1);   // P^T . dO, dS^T . Q
-            auto SdP = [&](int t) -> bool {
-                const int s = t % kStages;
-                if (!wait_bar(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
-                    return false;
-                if (!wait_bar(&s_empty[t & 1], ((t >> 1) & 1) ^ 1, abort_flag, status, wait_limit))
-                    return false;
-                tc_fence_after();
-                const uint32_t st = sb + KV_RING + s * kStageBytes;
+        // MMA issuer: whole warp, one elected lane issues
+        constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // K . Q^T, V . dO^T
+        constexpr uint32_t kIdG = idesc_bf16(128, 128, 0, 1);   // P^T . dO, dS^T . Q
+        auto SdP = [&](int t) -> bool {
+            const int s = t % kStages;
+            if (!warp_wait(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
+                return false;
+            if (!warp_wait(&s_empty[t & 1], ((t >> 1) & 1) ^ 1, abort_flag, status, wait_limit))
+                return false;
+            tc_fence_after();
+            const uint32_t st = sb + KV_RING + s * kStageBytes;
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                    const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_ss(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
-                           desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
-                    mma_ss(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
-                           desc_sw128(st + 16384 + kb, 16, 1024), kIdS, kk > 0);
-                }
-                mma_commit(&s_full[t & 1]);
-                return true;
-            };
-            auto Grad = [&](int t) -> bool {
-                const int s = t % kStages;
-                if (!wait_bar(pd_full, t & 1, abort_flag, status, wait_limit)) return false;
-                tc_fence_after();
-                const uint32_t st = sb + KV_RING + s * kStageBytes;
-#pragma unroll
-                for (int kk = 0; kk < 64 / 16; ++kk) {
-                    const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                    mma_ss(tmem + 256, desc_sw128(sb + KV_P + kk * 32, 16, 1024),
-                           desc_sw128(st + 16384 + kk * 2048, 8192, 1024), kIdG, acc);
-                    mma_ss(tmem + 384, desc_sw128(sb + KV_DS + kk * 32, 16, 1024),
-                           desc_sw128(st + kk * 2048, 8192, 1024), kIdG, acc);
-                }
-                mma_commit(pd_empty);
-                mma_commit(&st_empty[s]);
-                return true;
-            };
-            if (ntiles > 0 && wait_bar(kv_full, 0, abort_flag, status, wait_limit)) {
-                bool ok = SdP(0);
-                for (int t = 1; ok && t < ntiles; ++t) ok = SdP(t) && Grad(t - 1);
-                if (ok) Grad(ntiles - 1);
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_ss(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
+                       desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
+                mma_ss(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
+                       desc_sw128(st + 16384 + kb, 16, 1024), kIdS, kk > 0);
             }
-            mma_commit(done);
-            wait_plain(done, 0, wait_limit);
+            mma_commit(&s_full[t & 1]);
+            return true;
+        };
+        auto Grad = [&](int t) -> bool {
+            const int s = t % kStages;
+            if (!warp_wait(pd_full, t & 1, abort_flag, status, wait_limit)) return false;
+            tc_fence_after();
+            const uint32_t st = sb + KV_RING + s * kStageBytes;
+#pragma unroll
+            for (int kk = 0; kk < 64 / 16; ++kk) {
+                const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
+                mma_ss(tmem + 256, desc_sw128(sb + KV_P + kk * 32, 16, 1024),
+                       desc_sw128(st + 16384 + kk * 2048, 8192, 1024), kIdG, acc);
+                mma_ss(tmem + 384, desc_sw128(sb + KV_DS + kk * 32, 16, 1024),
+                       desc_sw128(st + kk * 2048, 8192, 1024), kIdG, acc);
+            }
+            mma_commit(pd_empty);
+            mma_commit(&st_empty[s]);
+            return true;
+        };
+        if (ntiles > 0 && warp_wait(kv_full, 0, abort_flag, status, wait_limit)) {
+            bool ok = SdP(0);
+            for (int t = 1; ok && t < ntiles; ++t) ok = SdP(t) && Grad(t - 1);
+            if (ok) Grad(ntiles - 1);
         }
+        mma_commit(done);
+        if (lane == 0) wait_plain(done, 0, wait_limit);
+        __syncwarp();
     } else if (warp >= 4) {
         const int wq = warp & 3;
         const int tw = wq * 32 + lane;  // key row 0..127
@@ -348,13 +348,16 @@ __global__ void __launch_bounds__(256, 1)
 // their mask rows one key block (64 keys) per tile:
 //   S  = Q . K^T,  dP = dO . V^T    (Q, dO are TMEM A operands; S, dP double-
 //                                    buffered in TMEM)
-//   dS = P (dP - D)  -> bf16, written over S in TMEM (one thread per query)
+//   dS = P (dP - D)  -> bf16, written over S in TMEM
 //   dQ += dS . K                     (dS the TMEM A operand, K from shared
 //                                    memory, MN-major; accumulator in TMEM)
+// dS has no reduction along a row, so two warpgroups share the work: thread
+// (g, r) handles query row r and keys [32 g, 32 g + 32) of the tile, and
+// writes their bf16 dS over its own S columns [32 g, 32 g + 16).
 // Queries of the pair whose own row does not keep a key block get dS = 0.
 // TMEM columns: buffer b in [128 b, 128 b + 128) holds S (64) then dP (64);
 // dQ [256, 384), Q [384, 448), dO [448, 512).
-constexpr int kDqThreads = 192;
+constexpr int kDqThreads = 320;
 constexpr int kDqRing = 6;
 constexpr uint32_t kDqSlot = 32768;  // K block 16 KB + V block 16 KB
 constexpr uint32_t kColDQ = 256, kColQ = 384, kColDO = 448;
@@ -384,7 +387,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t *uFlag = sm + DQ_UF;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + DQ_BAR);
     uint64_t *kv_full = bar, *kv_empty = bar + kDqRing, *s_full = bar + 2 * kDqRing;
-    // ds_full[t & 1]: the four dS warps wrote dS(t) (two barriers, so a warp
+    // ds_full[t & 1]: the eight dS warps wrote dS(t) (two barriers, so a warp
     // already on tile t+1 cannot complete tile t's phase for the others)
     uint64_t *ds_full = s_full + 2, *q_ready = ds_full + 2, *done = q_ready + 1;
     int *sInt = reinterpret_cast<int *>(sm + DQ_INT);  // [0] tmem base [1] tiles [2] abort
@@ -408,9 +411,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&ds_full[b], 4);
+            mbar_init(&ds_full[b], 8);
         }
-        mbar_init(q_ready, 4);
+        mbar_init(q_ready, 8);
         mbar_init(done, 1);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
@@ -465,64 +468,63 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         for (int u = t > kDqRing ? t - kDqRing : 0; u < t; ++u)
             wait_plain(&kv_full[u % kDqRing], (u / kDqRing) & 1, wait_limit);
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // Q . K^T, dO . V^T
-            constexpr uint32_t kIdQ = idesc_bf16(128, 128, 0, 1);   // dS . K (K MN-major)
-            auto SdP = [&](int t) -> bool {
-                const int slot = t % kDqRing;
-                if (!wait_bar(&kv_full[slot], (t / kDqRing) & 1, abort_flag, status, wait_limit))
-                    return false;
-                tc_fence_after();
-                const uint32_t b0 = sRing + slot * kDqSlot;
-                const uint32_t d = tmem + (t & 1) * 128;
+        // ---------------- MMA issuer (whole warp, one elected lane issues) ----------------
+        constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // Q . K^T, dO . V^T
+        constexpr uint32_t kIdQ = idesc_bf16(128, 128, 0, 1);   // dS . K (K MN-major)
+        auto SdP = [&](int t) -> bool {
+            const int slot = t % kDqRing;
+            if (!warp_wait(&kv_full[slot], (t / kDqRing) & 1, abort_flag, status, wait_limit))
+                return false;
+            tc_fence_after();
+            const uint32_t b0 = sRing + slot * kDqSlot;
+            const uint32_t d = tmem + (t & 1) * 128;
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                    mma_ts(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
-                    mma_ts(d + 64, tmem + kColDO + 8 * kk, desc_sw128(b0 + 16384 + off, 16, 1024),
-                           kIdS, kk > 0);
-                }
-                mma_commit(&s_full[t & 1]);
-                return true;
-            };
-            auto Grad = [&](int t) -> bool {
-                const int slot = t % kDqRing;
-                if (!wait_bar(&ds_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit))
-                    return false;
-                tc_fence_after();
-                const uint32_t b0 = sRing + slot * kDqSlot;
-#pragma unroll
-                for (int kk = 0; kk < 64 / 16; ++kk)
-                    mma_ts(tmem + kColDQ, tmem + (t & 1) * 128 + 8 * kk,
-                           desc_sw128(b0 + kk * 2048, 8192, 1024), kIdQ, (t > 0 || kk > 0));
-                mma_commit(&kv_empty[slot]);
-                return true;
-            };
-            if (ntiles > 0 && wait_bar(q_ready, 0, abort_flag, status, wait_limit)) {
-                bool ok = SdP(0);
-                for (int t = 0; ok && t < ntiles; ++t) {
-                    if (t + 1 < ntiles) ok = SdP(t + 1);
-                    ok = ok && Grad(t);
-                }
+            for (int kk = 0; kk < kD / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
+                mma_ts(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
+                mma_ts(d + 64, tmem + kColDO + 8 * kk, desc_sw128(b0 + 16384 + off, 16, 1024),
+                       kIdS, kk > 0);
             }
-            mma_commit(done);  // completes once every MMA issued above has finished
-            wait_plain(done, 0, wait_limit);
+            mma_commit(&s_full[t & 1]);
+            return true;
+        };
+        auto Grad = [&](int t) -> bool {
+            const int slot = t % kDqRing;
+            if (!warp_wait(&ds_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit))
+                return false;
+            tc_fence_after();
+            const uint32_t b0 = sRing + slot * kDqSlot;
+#pragma unroll
+            for (int kk = 0; kk < 64 / 16; ++kk)  // keys 16kk.. at column 32(kk/2) + 8(kk%2)
+                mma_ts(tmem + kColDQ, tmem + (t & 1) * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
+                       desc_sw128(b0 + kk * 2048, 8192, 1024), kIdQ, (t > 0 || kk > 0));
+            mma_commit(&kv_empty[slot]);
+            return true;
+        };
+        if (ntiles > 0 && warp_wait(q_ready, 0, abort_flag, status, wait_limit)) {
+            bool ok = SdP(0);
+            for (int t = 0; ok && t < ntiles; ++t) {
+                if (t + 1 < ntiles) ok = SdP(t + 1);
+                ok = ok && Grad(t);
+            }
         }
+        mma_commit(done);  // completes once every MMA issued above has finished
+        if (lane == 0) wait_plain(done, 0, wait_limit);
+        __syncwarp();
     } else if (warp >= 2) {
-        // ---------------- dS warpgroup: one thread per query row ----------------
+        // ---------------- dS warpgroups: query row r, key half kg ----------------
         const int wq = warp & 3;                    // TMEM lane quarter of this warp
+        const int kg = (warp - 2) >> 2;             // 0: keys 0-31, 1: keys 32-63
         const int r = wq * 32 + lane;               // query row of the pair, 0..127
         const int h = r >> 6;                       // 0 -> block iA, 1 -> block iB
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const int ib = h ? (iB >= 0 ? iB : iA) : iA;
         const int64_t grow = bh * N + static_cast<int64_t>(ib) * kBlk + (r & 63);
         const float Lr = l2[grow], Dr = dl[grow];
-        // Q and dO rows -> TMEM (the A operands of S and dP)
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-            const uint4 *src = reinterpret_cast<const uint4 *>((which ? dout : q) + grow * kD);
-            const uint32_t col = which ? kColDO : kColQ;
+        {
+            // Q (group 0) or dO (group 1) row -> TMEM, the A operands of S and dP
+            const uint4 *src = reinterpret_cast<const uint4 *>((kg ? dout : q) + grow * kD);
+            const uint32_t col = kg ? kColDO : kColQ;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t v32[32];
@@ -536,8 +538,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 }
                 tmem_st32(tmem + lane_base + col + 32 * half, reinterpret_cast<float *>(v32));
             }
+            tmem_wait_st();
         }
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(q_ready);
@@ -547,34 +549,31 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
             const bool valid = (uFlag[t] >> h) & 1u;  // uniform per warp
-            const uint32_t scol = tmem + lane_base + (t & 1) * 128;
-            uint32_t gk[32];
+            const uint32_t scol = tmem + lane_base + (t & 1) * 128 + 32 * kg;
+            uint32_t gk[16];
             if (valid) {
+                float sv[32], dp[32];
+                tmem_ld32(scol, sv);
+                tmem_ld32(scol + 64, dp);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float sv[32], dp[32];
-                    tmem_ld32(scol + 32 * half, sv);
-                    tmem_ld32(scol + 64 + 32 * half, dp);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float p0 = fast_exp2(fmaf(sv[e], c, -Lr));
-                        const float p1 = fast_exp2(fmaf(sv[e + 1], c, -Lr));
-                        gk[16 * half + (e >> 1)] = pack_bf16(p0 * (dp[e] - Dr), p1 * (dp[e + 1] - Dr));
-                    }
+                for (int e = 0; e < 32; e += 2) {
+                    const float p0 = fast_exp2(fmaf(sv[e], c, -Lr));
+                    const float p1 = fast_exp2(fmaf(sv[e + 1], c, -Lr));
+                    gk[e >> 1] = pack_bf16(p0 * (dp[e] - Dr), p1 * (dp[e + 1] - Dr));
                 }
             } else {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) gk[e] = 0u;
+                for (int e = 0; e < 16; ++e) gk[e] = 0u;
             }
-            // bf16 dS over the first 32 columns of this S buffer
-            tmem_st32(scol, reinterpret_cast<float *>(gk));
+            // bf16 dS of keys [32 kg, 32 kg + 32) over this group's first 16 S columns
+            tmem_st16(scol, gk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&ds_full[t & 1]);
         }
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue: group kg writes dQ features [64 kg, 64 kg + 64) ----------------
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
         // warp-uniform flags around the collective TMEM loads
@@ -582,12 +581,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const bool have = (h == 0 || iB >= 0) && !aborted;
         const bool live = have && ntiles > 0 && __all_sync(0xffffffffu, ok);
         if (have) {
-            __nv_bfloat16 *dst = dq + grow * kD;
+            __nv_bfloat16 *dst = dq + grow * kD + 64 * kg;
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
+            for (int part = 0; part < 2; ++part) {
                 float v[32];
                 if (live) {
-                    tmem_ld32(tmem + lane_base + kColDQ + 32 * part, v);
+                    tmem_ld32(tmem + lane_base + kColDQ + 64 * kg + 32 * part, v);
                     tmem_wait_ld();
                 } else {
 #pragma unroll

@@ -15,21 +15,25 @@
 //   S = Q_pair . K_tile^T   (M = 128 queries, N = 128 keys; Q is the TMEM
 //                            A operand, K the shared-memory B operand;
 //                            S double-buffered in TMEM)
-//   P = exp2(S * scale*log2e - m)   one softmax thread per query row: the
-//                            row maximum and sum are thread-local; bf16 P is
-//                            written back over S in TMEM
+//   P = exp2(S * scale*log2e - m)   two softmax warpgroups: thread (g, r)
+//                            owns query row r and the 64 keys of union block
+//                            2t+g; the row maximum is combined through shared
+//                            memory; bf16 P is written back over S in TMEM
 //   O += P . V_tile          (P the TMEM A operand, V from shared memory)
 // Each row keeps a reference maximum m; when a tile's maximum exceeds it by
-// more than 2^8 the row moves to the new maximum and rescales its own O row
-// in TMEM and its sum (the exponent never exceeds 2^8 otherwise).
+// more than 2^8 the row moves to the new maximum and both halves rescale
+// their half of the O row in TMEM and their partial sums (the exponent never
+// exceeds 2^8 otherwise).
 //
-// Warp roles (192 threads): warp 0 builds the union list (OR of the two
+// Warp roles (320 threads): warp 0 builds the union list (OR of the two
 // bit rows) and issues TMA loads of K and V through a 6-slot ring in MMA
-// consumption order (K0 K1 V0 K2 V1 ...); warp 1 owns TMEM and issues the
-// MMAs (S(t+1) before O += P(t) V(t), so the next scores are computed while
-// this tile's softmax runs); warps 2-5 are the softmax warpgroup (thread =
-// query row; warp w serves TMEM lane quarter w % 4).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), Q [384,448).
+// consumption order (K0 K1 V0 K2 V1 ...); warp 1 owns TMEM and one of its
+// threads issues the MMAs (S(t+1) before O += P(t) V(t), so the next scores
+// are computed while this tile's softmax runs); warps 2-9 are the softmax
+// warpgroups (warp w serves TMEM lane quarter w % 4 and key half (w - 2) / 4).
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), Q [384,448).  Key half
+// g of a tile has its scores in columns [64 g, 64 g + 64) of the S buffer and
+// its bf16 P in the first 32 of them.
 // Every wait is bounded: on expiry the CTA records a timeout in the status
 // word, unwinds without further work, drains its in-flight copies and MMAs
 // and frees TMEM; later CTAs of the launch see the status and do nothing.
@@ -40,7 +44,7 @@ namespace fwd100 {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kRing = 6;
 constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 bf16
 constexpr int kD = 128;
@@ -54,7 +58,9 @@ constexpr uint32_t OFF_RING = 0;                                  // kRing x 32 
 constexpr uint32_t OFF_U = OFF_RING + kRing * kTileBytes;         // union list u16
 constexpr uint32_t OFF_UF = OFF_U + 2 * (kMaxNbFwd + 8);          // membership per entry
 constexpr uint32_t OFF_TM = OFF_UF + kMaxNbFwd + 8;               // membership per tile
-constexpr uint32_t OFF_BAR = ((OFF_TM + kMaxNbFwd / 2 + 8 + 7) / 8) * 8;
+// [3][2][128] f32: partial row maxima by tile parity, then the partial sums
+constexpr uint32_t OFF_RED = ((OFF_TM + kMaxNbFwd / 2 + 8 + 15) / 16) * 16;
+constexpr uint32_t OFF_BAR = OFF_RED + 3 * 2 * 128 * 4;
 constexpr int kNumBars = 2 * kRing + 2 + 1 + 2 + 1 + 1 + 1;
 constexpr uint32_t OFF_INT = OFF_BAR + 8 * kNumBars;              // ints
 constexpr uint32_t kSmemBytes = OFF_INT + 16 + 1024;              // + alignment slack
@@ -74,10 +80,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *tileMem = sm + OFF_TM;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *kv_full = bar, *kv_empty = bar + kRing, *s_full = bar + 2 * kRing;
-    // p_full[t & 1]: the four softmax warps wrote P(t).  Two barriers, so that a
+    // p_full[t & 1]: the eight softmax warps wrote P(t).  Two barriers, so that a
     // warp already on tile t+1 cannot complete tile t's phase for the others.
     uint64_t *q_ready = s_full + 2, *p_full = q_ready + 1, *p_empty = p_full + 2;
     uint64_t *o_done = p_empty + 1, *never = o_done + 1;
+    float *red = reinterpret_cast<float *>(sm + OFF_RED);  // [slot][half][row]
     int *sInt = reinterpret_cast<int *>(sm + OFF_INT);  // [0] tmem base [1] tiles [2] abort
     volatile int *abort_flag = sInt + 2;
 
@@ -99,9 +106,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(q_ready, 4);
-        mbar_init(&p_full[0], 4);
-        mbar_init(&p_full[1], 4);
+        mbar_init(q_ready, 8);
+        mbar_init(&p_full[0], 8);
+        mbar_init(&p_full[1], 8);
         mbar_init(p_empty, 1);
         mbar_init(o_done, 1);
         mbar_init(never, 1);
@@ -163,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (uint32_t s = seq > kRing ? seq - kRing : 0; s < seq; ++s)
             wait_plain(&kv_full[s % kRing], (s / kRing) & 1u, wait_limit);
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
+        // ---------------- MMA issuer (one thread) ----------------
         if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);   // Q . K^T
             constexpr uint32_t kIdPV = idesc_bf16(128, 128, 0, 1);  // P . V (V MN-major)
@@ -177,10 +184,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d = tmem + (t & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk)
-                    mma_ts(d, tmem + kColQ + 8 * kk,
-                           desc_sw128(b0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
-                mma_commit(&kv_empty[slot]);
-                mma_commit(&s_full[t & 1]);
+                    mma_ts_1(d, tmem + kColQ + 8 * kk,
+                             desc_sw128(b0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), kIdS,
+                             kk > 0);
+                mma_commit_1(&kv_empty[slot]);
+                mma_commit_1(&s_full[t & 1]);
                 ++seq;
                 return true;
             };
@@ -194,11 +202,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t b0 = sRing + slot * kTileBytes;
                 const uint32_t pcol = tmem + (t & 1) * 128;
 #pragma unroll
-                for (int kk = 0; kk < 128 / 16; ++kk)
-                    mma_ts(tmem + kColO, pcol + 8 * kk, desc_sw128(b0 + kk * 2048, 16384, 1024),
-                           kIdPV, (t > 0 || kk > 0));
-                mma_commit(&kv_empty[slot]);
-                mma_commit(p_empty);
+                for (int kk = 0; kk < 128 / 16; ++kk)  // keys 16kk.. at column 64(kk/4) + 8(kk%4)
+                    mma_ts_1(tmem + kColO, pcol + 64 * (kk >> 2) + 8 * (kk & 3),
+                             desc_sw128(b0 + kk * 2048, 16384, 1024), kIdPV, (t > 0 || kk > 0));
+                mma_commit_1(&kv_empty[slot]);
+                mma_commit_1(p_empty);
                 ++seq;
                 return true;
             };
@@ -209,12 +217,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = ok && PV(t);
                 }
             }
-            mma_commit(o_done);  // completes once every MMA issued above has finished
+            mma_commit_1(o_done);  // completes once every MMA issued above has finished
             wait_plain(o_done, 0, wait_limit);
         }
     } else if (warp >= 2) {
-        // ---------------- softmax warpgroup: one thread per query row ----------------
+        // ---------------- softmax: thread (g, r) = key half g, query row r ----------------
         const int wq = warp & 3;                    // TMEM lane quarter of this warp
+        const int g = (warp - 2) >> 2;              // key half of the tile
         const int r = wq * 32 + lane;               // query row of the pair, 0..127
         const int h = r >> 6;                       // 0 -> block iA, 1 -> block iB
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
@@ -222,102 +231,104 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t grow = bh * N + static_cast<int64_t>(ib) * kBlk + (r & 63);
         bool ok = true;
         if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
-        // Q row -> TMEM (the A operand of S = Q K^T)
         {
-            const uint4 *src = reinterpret_cast<const uint4 *>(q + grow * kD);
+            // features [64 g, 64 g + 64) of the Q row -> TMEM (the A operand of S = Q K^T)
+            const uint4 *src = reinterpret_cast<const uint4 *>(q + grow * kD + 64 * g);
             uint32_t qv[32];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const uint4 v = __ldg(src + 8 * half + e);
-                    qv[4 * e] = v.x;
-                    qv[4 * e + 1] = v.y;
-                    qv[4 * e + 2] = v.z;
-                    qv[4 * e + 3] = v.w;
-                }
-                tmem_st32(tmem + lane_base + kColQ + 32 * half, reinterpret_cast<float *>(qv));
+            for (int e = 0; e < 8; ++e) {
+                const uint4 v = __ldg(src + e);
+                qv[4 * e] = v.x;
+                qv[4 * e + 1] = v.y;
+                qv[4 * e + 2] = v.z;
+                qv[4 * e + 3] = v.w;
             }
+            tmem_st32(tmem + lane_base + kColQ + 32 * g, reinterpret_cast<float *>(qv));
             tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(q_ready);
 
-        float m = -INFINITY, l = 0.f;
+        float m = -INFINITY, l = 0.f;  // l: partial sum over this half's keys
         for (int t = 0; t < ntiles; ++t) {
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
-            const uint32_t mem = tileMem[t];
-            const bool va = (mem >> h) & 1u, vb = (mem >> (2 + h)) & 1u;
-            const uint32_t scol = tmem + lane_base + (t & 1) * 128;
-            uint32_t pk[64];
-            if (!(va || vb)) {
-#pragma unroll
-                for (int e = 0; e < 64; ++e) pk[e] = 0u;
-            } else {
-                float s[128];
-#pragma unroll
-                for (int part = 0; part < 4; ++part) tmem_ld32(scol + 32 * part, s + 32 * part);
+            const bool valid = (tileMem[t] >> (2 * g + h)) & 1u;  // uniform per warp
+            const uint32_t scol = tmem + lane_base + (t & 1) * 128 + 64 * g;
+            float s[64];
+            float pmax = -INFINITY;
+            if (valid) {
+                tmem_ld32(scol, s);
+                tmem_ld32(scol + 32, s + 32);
                 tmem_wait_ld();
                 float mx8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+                for (int e = 0; e < 8; ++e) mx8[e] = s[e];
 #pragma unroll
-                for (int k = 0; k < 128; ++k) {
-                    const bool vk = k < 64 ? va : vb;
-                    s[k] = vk ? s[k] : -INFINITY;
-                    mx8[k & 7] = fmaxf(mx8[k & 7], s[k]);
-                }
-                const float tmax = c * fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                // TMEM loads/stores are warp-collective (.sync.aligned): the
-                // decision to move to a new reference is taken per warp; every
-                // lane then moves to max(m, tmax), which is exact for all rows.
-                if (__any_sync(0xffffffffu, tmax > m + kRescaleAt)) {
-                    const float mnew = fmaxf(m, tmax);
-                    const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mnew);
-                    if (__any_sync(0xffffffffu, m != -INFINITY)) {
-                        // rows with earlier keys: O and the sum move to mnew
-                        ok = wait_bar(p_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
-                        tc_fence_after();
+                for (int k = 8; k < 64; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], s[k]);
+                pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            }
+            // row maximum over both halves
+            red[((t & 1) * 2 + g) * 128 + r] = pmax;
+            bar_sync(1, 256);
+            const float tmax = c * fmaxf(pmax, red[((t & 1) * 2 + (g ^ 1)) * 128 + r]);
+            // TMEM loads/stores are warp-collective (.sync.aligned): the
+            // decision to move to a new reference is taken per warp (the two
+            // warps serving the same rows take the same decision from the same
+            // values); every lane then moves to max(m, tmax).
+            if (__any_sync(0xffffffffu, tmax > m + kRescaleAt)) {
+                const float mnew = fmaxf(m, tmax);
+                const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mnew);
+                if (__any_sync(0xffffffffu, m != -INFINITY)) {
+                    // rows with earlier keys: this half of the O row moves to mnew
+                    ok = wait_bar(p_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
+                    tc_fence_after();
 #pragma unroll
-                        for (int part = 0; part < 4; ++part) {
-                            float ov[32];
-                            tmem_ld32(tmem + lane_base + kColO + 32 * part, ov);
-                            tmem_wait_ld();
+                    for (int part = 0; part < 2; ++part) {
+                        float ov[32];
+                        tmem_ld32(tmem + lane_base + kColO + 64 * g + 32 * part, ov);
+                        tmem_wait_ld();
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-                            tmem_st32(tmem + lane_base + kColO + 32 * part, ov);
-                        }
-                        tmem_wait_st();
+                        for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                        tmem_st32(tmem + lane_base + kColO + 64 * g + 32 * part, ov);
                     }
-                    l *= alpha;
-                    m = mnew;
+                    tmem_wait_st();
                 }
+                l *= alpha;
+                m = mnew;
+            }
+            uint32_t pk[32];
+            if (valid) {
                 float ls8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
 #pragma unroll
-                for (int k = 0; k < 128; k += 2) {
+                for (int k = 0; k < 64; k += 2) {
                     const float p0 = fast_exp2(fmaf(s[k], c, -m));
                     const float p1 = fast_exp2(fmaf(s[k + 1], c, -m));
                     ls8[(k >> 1) & 7] += p0 + p1;
                     pk[k >> 1] = pack_bf16(p0, p1);
                 }
                 l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) pk[e] = 0u;
             }
-            // bf16 P over the first 64 columns of this S buffer
+            // bf16 P over the first 32 columns of this half's scores
             tmem_st32(scol, reinterpret_cast<float *>(pk));
-            tmem_st32(scol + 32, reinterpret_cast<float *>(pk + 32));
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[t & 1]);
         }
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue: half g writes features [64 g, 64 g + 64) ----------------
         if (ok && ntiles > 0) ok = wait_bar(o_done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
+        red[(4 + g) * 128 + r] = l;  // own slot: the partner may still read the last maxima
+        bar_sync(1, 256);
+        l += red[(4 + (g ^ 1)) * 128 + r];
         // warp-uniform: every lane of the warp takes the same branches around
         // the collective TMEM loads
         const bool aborted = __any_sync(0xffffffffu, *abort_flag != 0);
@@ -325,14 +336,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool read_o = have && ntiles > 0 && __all_sync(0xffffffffu, ok);
         if (have) {
             const bool live = read_o && l > 0.f;
-            if (lse != nullptr) lse[grow] = live ? (m + log2f(l)) * kLn2 : -INFINITY;
+            if (lse != nullptr && g == 0) lse[grow] = live ? (m + log2f(l)) * kLn2 : -INFINITY;
             const float inv = live ? 1.f / l : 0.f;
-            __nv_bfloat16 *dst = out + grow * kD;
+            __nv_bfloat16 *dst = out + grow * kD + 64 * g;
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
+            for (int part = 0; part < 2; ++part) {
                 float ov[32];
                 if (read_o) {
-                    tmem_ld32(tmem + lane_base + kColO + 32 * part, ov);
+                    tmem_ld32(tmem + lane_base + kColO + 64 * g + 32 * part, ov);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
