@@ -11,8 +11,10 @@
 //   rows on the M = 128 datapath), walking the union of their mask columns,
 //   one query block (64 queries) per tile:
 //     S^T  = K . Q^T,  dP^T = V . dO^T                 (TMEM, double-buffered)
-//     P^T, dS^T = P^T (dP^T - D)  -> bf16, shared memory (one thread per key)
-//     dV  += P^T . dO,  dK += dS^T . Q                  (TMEM accumulators)
+//     P^T, dS^T = P^T (dP^T - D)  -> bf16 over S^T, dP^T in TMEM (two
+//                                    warpgroups, 32 queries each)
+//     dV  += P^T . dO,  dK += dS^T . Q                  (TMEM A operands and
+//                                                        accumulators)
 // dq_kernel: one CTA per pair of temporally adjacent QUERY blocks (128 query
 //   rows), walking the union of their mask rows, one key block per tile:
 //     S = Q . K^T,  dP = dO . V^T     (Q, dO resident in TMEM as A operands)
@@ -66,20 +68,23 @@ __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restric
 // dK, dV
 // ---------------------------------------------------------------------------
 constexpr int kStages = 3;
+constexpr int kKvThreads = 320;
 constexpr uint32_t kStageBytes = 33792;  // Q 16 KB + dO 16 KB + L2 256 B + D 256 B (+ pad)
 constexpr uint32_t KV_K = 0, KV_V = 32768;
 constexpr uint32_t KV_RING = 65536;
-constexpr uint32_t KV_P = KV_RING + kStages * kStageBytes;  // P^T 16 KB
-constexpr uint32_t KV_DS = KV_P + 16384;                    // dS^T 16 KB
-constexpr uint32_t KV_U = KV_DS + 16384;                    // union list
+constexpr uint32_t KV_U = KV_RING + kStages * kStageBytes;  // union list
 constexpr uint32_t KV_UF = KV_U + 2 * (kMaxNbBwd + 8);
 constexpr uint32_t KV_CB = ((KV_UF + kMaxNbBwd + 8 + 15) / 16) * 16;  // column bits [2][64]
 constexpr uint32_t KV_BAR = KV_CB + 2 * 256;
-constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 1;
+constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1;
 constexpr uint32_t KV_INT = KV_BAR + 8 * kKvBars;
 constexpr uint32_t kKvSmem = KV_INT + 16 + 1024;
 
-__global__ void __launch_bounds__(256, 1)
+// TMEM columns: S^T(t) [64 (t&1), +64), dP^T(t) [128 + 64 (t&1), +64),
+// dV [256, 384), dK [384, 512).  Warpgroup qg handles queries [32 qg, +32) of
+// the tile and writes bf16 P^T and dS^T for them over the first 16 of its
+// own S^T and dP^T columns, where the dV and dK MMAs read them.
+__global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                 const float *__restrict__ l2, const float *__restrict__ dl,
@@ -97,8 +102,9 @@ __global__ void __launch_bounds__(256, 1)
     uint32_t *colBits = reinterpret_cast<uint32_t *>(sm + KV_CB);  // [2][64 words]
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + KV_BAR);
     uint64_t *kv_full = bar, *st_full = bar + 1, *st_empty = bar + 1 + kStages;
-    uint64_t *s_full = bar + 1 + 2 * kStages, *s_empty = s_full + 2, *pd_full = s_empty + 2;
-    uint64_t *pd_empty = pd_full + 1, *done = pd_empty + 1;
+    // pd_full[t & 1]: the eight softmax warps wrote P^T(t), dS^T(t) (two
+    // barriers, so a warp already on tile t+1 cannot complete tile t's phase)
+    uint64_t *s_full = bar + 1 + 2 * kStages, *pd_full = s_full + 2, *done = pd_full + 2;
     int *sInt = reinterpret_cast<int *>(sm + KV_INT);
     volatile int *abort_flag = sInt + 2;
 
@@ -121,10 +127,8 @@ __global__ void __launch_bounds__(256, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&s_empty[b], 4);
+            mbar_init(&pd_full[b], 8);
         }
-        mbar_init(pd_full, 4);
-        mbar_init(pd_empty, 1);
         mbar_init(done, 1);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
@@ -156,7 +160,6 @@ __global__ void __launch_bounds__(256, 1)
     tc_fence_after();
     const uint32_t tmem = static_cast<uint32_t>(sInt[0]);
     const int ntiles = *abort_flag ? 0 : sInt[1];  // one query block per tile
-    // TMEM columns: S^T [0,128) (2 x 64), dP^T [128,256) (2 x 64), dV [256,384), dK [384,512)
 
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tq);
@@ -197,106 +200,96 @@ __global__ void __launch_bounds__(256, 1)
             const int s = t % kStages;
             if (!warp_wait(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
                 return false;
-            if (!warp_wait(&s_empty[t & 1], ((t >> 1) & 1) ^ 1, abort_flag, status, wait_limit))
-                return false;
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
                 const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
                 const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_ss(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
-                       desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
-                mma_ss(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
-                       desc_sw128(st + 16384 + kb, 16, 1024), kIdS, kk > 0);
+                mma_ss_warp(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
+                            desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
+                mma_ss_warp(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
+                            desc_sw128(st + 16384 + kb, 16, 1024), kIdS, kk > 0);
             }
-            mma_commit(&s_full[t & 1]);
+            mma_commit_warp(&s_full[t & 1]);
             return true;
         };
         auto Grad = [&](int t) -> bool {
             const int s = t % kStages;
-            if (!warp_wait(pd_full, t & 1, abort_flag, status, wait_limit)) return false;
+            if (!warp_wait(&pd_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit))
+                return false;
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
 #pragma unroll
-            for (int kk = 0; kk < 64 / 16; ++kk) {
+            for (int kk = 0; kk < 64 / 16; ++kk) {  // queries 16kk.. at column 32(kk/2) + 8(kk%2)
                 const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                mma_ss(tmem + 256, desc_sw128(sb + KV_P + kk * 32, 16, 1024),
-                       desc_sw128(st + 16384 + kk * 2048, 8192, 1024), kIdG, acc);
-                mma_ss(tmem + 384, desc_sw128(sb + KV_DS + kk * 32, 16, 1024),
-                       desc_sw128(st + kk * 2048, 8192, 1024), kIdG, acc);
+                const uint32_t col = (t & 1) * 64 + 32 * (kk >> 1) + 8 * (kk & 1);
+                mma_ts_warp(tmem + 256, tmem + col, desc_sw128(st + 16384 + kk * 2048, 8192, 1024),
+                            kIdG, acc);
+                mma_ts_warp(tmem + 384, tmem + 128 + col, desc_sw128(st + kk * 2048, 8192, 1024),
+                            kIdG, acc);
             }
-            mma_commit(pd_empty);
-            mma_commit(&st_empty[s]);
+            mma_commit_warp(&st_empty[s]);
             return true;
         };
         if (ntiles > 0 && warp_wait(kv_full, 0, abort_flag, status, wait_limit)) {
             bool ok = SdP(0);
-            for (int t = 1; ok && t < ntiles; ++t) ok = SdP(t) && Grad(t - 1);
-            if (ok) Grad(ntiles - 1);
+            for (int t = 0; ok && t < ntiles; ++t) {
+                if (t + 1 < ntiles) ok = SdP(t + 1);
+                ok = ok && Grad(t);
+            }
         }
-        mma_commit(done);
+        mma_commit_warp(done);
         if (lane == 0) wait_plain(done, 0, wait_limit);
         __syncwarp();
-    } else if (warp >= 4) {
+    } else if (warp >= 2) {
         const int wq = warp & 3;
-        const int tw = wq * 32 + lane;  // key row 0..127
-        const int kh = tw >> 6;         // key block of the pair
+        const int qg = (warp - 2) >> 2;  // queries [32 qg, 32 qg + 32) of each tile
+        const int tw = wq * 32 + lane;   // key row 0..127
+        const int kh = tw >> 6;          // key block of the pair
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
-            const bool valid = (uFlag[t] >> kh) & 1u;
-            const int s = t % kStages;
-            const float *L = reinterpret_cast<const float *>(sm + KV_RING + s * kStageBytes + 32768);
-            const float *Dv = L + 64;
-            uint32_t pk[32], dk2[32];  // packed bf16 pairs of P^T and dS^T rows
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            const bool valid = (uFlag[t] >> kh) & 1u;  // uniform per warp
+            const uint32_t scol = tmem + lane_base + (t & 1) * 64 + 32 * qg;
+            uint32_t pk[16], dk2[16];  // packed bf16 pairs of P^T and dS^T
+            if (valid) {
+                const float4 *L4 = reinterpret_cast<const float4 *>(
+                    sm + KV_RING + (t % kStages) * kStageBytes + 32768 + 128 * qg);
+                const float4 *D4 = L4 + 16;  // D follows L2 at +256 bytes
                 float sv[32], dp[32];
-                tmem_ld32(tmem + lane_base + (t & 1) * 64 + 32 * half, sv);
-                tmem_ld32(tmem + lane_base + 128 + (t & 1) * 64 + 32 * half, dp);
+                tmem_ld32(scol, sv);
+                tmem_ld32(scol + 128, dp);
                 tmem_wait_ld();
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) {
-                    const float4 l4 = reinterpret_cast<const float4 *>(L)[8 * half + q4];
-                    const float4 d4 = reinterpret_cast<const float4 *>(Dv)[8 * half + q4];
+                    const float4 l4 = L4[q4], d4 = D4[q4];
                     const float la[4] = {l4.x, l4.y, l4.z, l4.w};
                     const float da[4] = {d4.x, d4.y, d4.z, d4.w};
                     float pv[4], gv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int q = 4 * q4 + e;
-                        pv[e] = valid ? fast_exp2(fmaf(sv[q], c, -la[e])) : 0.f;
+                        pv[e] = fast_exp2(fmaf(sv[q], c, -la[e]));
                         gv[e] = pv[e] * (dp[q] - da[e]);
                     }
-                    pk[16 * half + 2 * q4] = pack_bf16(pv[0], pv[1]);
-                    pk[16 * half + 2 * q4 + 1] = pack_bf16(pv[2], pv[3]);
-                    dk2[16 * half + 2 * q4] = pack_bf16(gv[0], gv[1]);
-                    dk2[16 * half + 2 * q4 + 1] = pack_bf16(gv[2], gv[3]);
+                    pk[2 * q4] = pack_bf16(pv[0], pv[1]);
+                    pk[2 * q4 + 1] = pack_bf16(pv[2], pv[3]);
+                    dk2[2 * q4] = pack_bf16(gv[0], gv[1]);
+                    dk2[2 * q4 + 1] = pack_bf16(gv[2], gv[3]);
                 }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) pk[e] = dk2[e] = 0u;
             }
+            tmem_st16(scol, pk);
+            tmem_st16(scol + 128, dk2);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&s_empty[t & 1]);
-            if (t > 0) ok = wait_bar(pd_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
-            const uint32_t prow = sb + KV_P + tw * 128, drow = sb + KV_DS + tw * 128;
-#pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const uint32_t off = (cc ^ (tw & 7)) << 4;
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(prow + off),
-                             "r"(pk[4 * cc]), "r"(pk[4 * cc + 1]), "r"(pk[4 * cc + 2]),
-                             "r"(pk[4 * cc + 3])
-                             : "memory");
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};\n" ::"r"(drow + off),
-                             "r"(dk2[4 * cc]), "r"(dk2[4 * cc + 1]), "r"(dk2[4 * cc + 2]),
-                             "r"(dk2[4 * cc + 3])
-                             : "memory");
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(pd_full);
+            if (lane == 0) mbar_arrive(&pd_full[t & 1]);
         }
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
@@ -305,31 +298,29 @@ __global__ void __launch_bounds__(256, 1)
         const bool all_ok = __all_sync(0xffffffffu, ok);
         const int jm = kh ? jB : jA;
         if (jm >= 0 && !aborted) {
+            // warpgroup 0 writes the dV row, warpgroup 1 the dK row of key tw
             const int64_t row = bh * N + static_cast<int64_t>(jm) * kBlk + (tw & 63);
             const bool live = all_ok && ntiles > 0;
+            __nv_bfloat16 *dst = (qg ? dk : dv) + row * kD;
+            const float mul = qg ? scale : 1.f;
 #pragma unroll
-            for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
-                __nv_bfloat16 *dst = (which ? dk : dv) + row * kD;
-                const float mul = which ? scale : 1.f;
+            for (int part = 0; part < 4; ++part) {
+                float v[32];
+                if (live) {
+                    tmem_ld32(tmem + lane_base + 256 + 128 * qg + 32 * part, v);
+                    tmem_wait_ld();
+                } else {
 #pragma unroll
-                for (int part = 0; part < 4; ++part) {
-                    float v[32];
-                    if (live) {
-                        tmem_ld32(tmem + lane_base + 256 + 128 * which + 32 * part, v);
-                        tmem_wait_ld();
-                    } else {
+                    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+                }
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = 0.f;
-                    }
-#pragma unroll
-                    for (int e8 = 0; e8 < 4; ++e8) {
-                        uint4 w;
-                        w.x = pack_bf16(v[8 * e8] * mul, v[8 * e8 + 1] * mul);
-                        w.y = pack_bf16(v[8 * e8 + 2] * mul, v[8 * e8 + 3] * mul);
-                        w.z = pack_bf16(v[8 * e8 + 4] * mul, v[8 * e8 + 5] * mul);
-                        w.w = pack_bf16(v[8 * e8 + 6] * mul, v[8 * e8 + 7] * mul);
-                        *reinterpret_cast<uint4 *>(dst + 32 * part + 8 * e8) = w;
-                    }
+                for (int e8 = 0; e8 < 4; ++e8) {
+                    uint4 w;
+                    w.x = pack_bf16(v[8 * e8] * mul, v[8 * e8 + 1] * mul);
+                    w.y = pack_bf16(v[8 * e8 + 2] * mul, v[8 * e8 + 3] * mul);
+                    w.z = pack_bf16(v[8 * e8 + 4] * mul, v[8 * e8 + 5] * mul);
+                    w.w = pack_bf16(v[8 * e8 + 6] * mul, v[8 * e8 + 7] * mul);
+                    *reinterpret_cast<uint4 *>(dst + 32 * part + 8 * e8) = w;
                 }
             }
         }
@@ -481,11 +472,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_ts(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
-                mma_ts(d + 64, tmem + kColDO + 8 * kk, desc_sw128(b0 + 16384 + off, 16, 1024),
+                mma_ts_warp(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
+                mma_ts_warp(d + 64, tmem + kColDO + 8 * kk, desc_sw128(b0 + 16384 + off, 16, 1024),
                        kIdS, kk > 0);
             }
-            mma_commit(&s_full[t & 1]);
+            mma_commit_warp(&s_full[t & 1]);
             return true;
         };
         auto Grad = [&](int t) -> bool {
@@ -496,9 +487,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const uint32_t b0 = sRing + slot * kDqSlot;
 #pragma unroll
             for (int kk = 0; kk < 64 / 16; ++kk)  // keys 16kk.. at column 32(kk/2) + 8(kk%2)
-                mma_ts(tmem + kColDQ, tmem + (t & 1) * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
+                mma_ts_warp(tmem + kColDQ, tmem + (t & 1) * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
                        desc_sw128(b0 + kk * 2048, 8192, 1024), kIdQ, (t > 0 || kk > 0));
-            mma_commit(&kv_empty[slot]);
+            mma_commit_warp(&kv_empty[slot]);
             return true;
         };
         if (ntiles > 0 && warp_wait(q_ready, 0, abort_flag, status, wait_limit)) {
@@ -508,7 +499,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 ok = ok && Grad(t);
             }
         }
-        mma_commit(done);  // completes once every MMA issued above has finished
+        mma_commit_warp(done);  // completes once every MMA issued above has finished
         if (lane == 0) wait_plain(done, 0, wait_limit);
         __syncwarp();
     } else if (warp >= 2) {
@@ -637,7 +628,7 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
                                static_cast<int>(kKvSmem));
     if (err != cudaSuccess) return err;
     const int64_t groups = static_cast<int64_t>((T + 1) / 2) * Hp * Wp;
-    dkdv_kernel<<<static_cast<unsigned>(BH * groups), 256, kKvSmem, stream>>>(
+    dkdv_kernel<<<static_cast<unsigned>(BH * groups), kKvThreads, kKvSmem, stream>>>(
         mq, mk, mv, mdo, l2, dl, col_idx, col_cnt, static_cast<__nv_bfloat16 *>(dk),
         static_cast<__nv_bfloat16 *>(dv), status, nb, Hp, Wp, T, c, scale, limit);
     err = cudaGetLastError();

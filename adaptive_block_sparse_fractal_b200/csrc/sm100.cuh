@@ -95,13 +95,14 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 }
-// MMA issue is warp-collective: the whole warp executes the call, converged,
-// and one elected lane issues the instruction.  Keeping the issuing code
+// *_warp: MMA issue is warp-collective: the whole warp executes the call,
+// converged, and one elected lane issues the instruction (calling one from a
+// single lane deadlocks the warp).  Keeping the issuing code
 // convergent lets the descriptors live in uniform registers; issuing from a
 // single divergent lane costs more than an N = 64 MMA takes to execute.
 //
 // D[tmem] (+)= A[smem] * B[smem], kind::f16 (bf16 inputs, fp32 accumulate).
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n .reg .pred e, p;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
@@ -110,7 +111,7 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t
 }
 // D[tmem] (+)= A[tmem] * B[smem], kind::f16; A is M x K, K-major, 16-bit
 // elements packed two per 32-bit column (a K = 16 step spans 8 columns).
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+__device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
                                        uint32_t idesc, uint32_t accumulate) {
     asm volatile(
         "{\n .reg .pred e, p;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p, %4, 0;\n"
@@ -135,7 +136,7 @@ __device__ __forceinline__ void mma_commit_1(uint64_t *bar) {
 }
 // Arrive on `bar` once all previously issued tcgen05 ops of the issuing
 // thread are done (warp-collective, one elected lane commits).
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+__device__ __forceinline__ void mma_commit_warp(uint64_t *bar) {
     asm volatile(
         "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
         " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(
