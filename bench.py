@@ -36,6 +36,16 @@ WORKLOAD = "train"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, per
+# head, from one ncu --set full capture of `bench.py --heads 8` (same shape,
+# 8 heads; heads are independent, so the traffic scales with their number).
+# Must be re-measured whenever these kernels change.
+NCU_DRAM_BYTES_PER_HEAD = {
+    ("train", "attn_bwd"): (324.7e6 + 956.0e6 + 792.7e6) / 8,  # pre + dK/dV + dQ
+    ("train", "attn_fwd"): (476.3e6 + 146.1e6) / 8,
+}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -318,8 +328,12 @@ def run_nabla(args):
     dom = max(ops, key=lambda k: ops[k][0])
     achieved = ops[dom][1] / (ops[dom][0] * 1e-3) / 1e12
     peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = None
+    per_head = NCU_DRAM_BYTES_PER_HEAD.get((args.workload, dom))
+    if per_head is not None:
+        traffic = per_head * w.heads
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dom,
+                "frac": achieved / peak, "traffic": traffic, "kernel": dom,
                 "peak_source": "bf16 sustained (of %s)" % pk_src,
                 "flop_per_launch": ops[dom][1], "ms_per_launch": ops[dom][0],
                 "frac_of_burst": achieved / pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])}
