@@ -15,7 +15,8 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, f
                                     float scale, int wt, int wh, int ww, unsigned flags,
                                     const void *q, const void *k, float *qbar, float *kbar_t,
                                     uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
-                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream);
+                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream,
+                                    const void *q_grid, const void *k_grid);
 cudaError_t nabla_launch_attn_fwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
                                       const void *k, const void *v, const uint16_t *row_idx,
                                       const int32_t *row_cnt, void *o, float *lse,
@@ -186,7 +187,49 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params, const
     return cuda_status(nabla_launch_build_mask(
         d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
         params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
-        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr, s));
+        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr, s,
+        nullptr, nullptr));
+}
+
+namespace {
+bool overlap(const void *a, const void *b, size_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+}  // namespace
+
+int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
+                          const nabla_bf16 *q_grid, const nabla_bf16 *k_grid, nabla_bf16 *q,
+                          nabla_bf16 *k, const nabla_mask *mask, void *workspace,
+                          size_t workspace_bytes, nabla_stream_t stream) {
+    Dims d;
+    int st = check_shape(shape, &d);
+    if (st != NABLA_OK) return st;
+    if ((st = check_params(params, true)) != NABLA_OK) return st;
+    if (q_grid == nullptr || k_grid == nullptr || q == nullptr || k == nullptr ||
+        mask == nullptr || mask->bits == nullptr || mask->row_idx == nullptr ||
+        mask->row_cnt == nullptr)
+        return NABLA_ERR_NULL;
+    const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
+    if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
+    if (!aligned16(q_grid) || !aligned16(k_grid) || !aligned16(q) || !aligned16(k))
+        return NABLA_ERR_ALIGN;
+    // the flattened outputs must not overlap each other or either input
+    const size_t bytes = sizeof(nabla_bf16) * static_cast<size_t>(d.BH) * d.N * d.D;
+    if (overlap(q, k, bytes) || overlap(q, q_grid, bytes) || overlap(q, k_grid, bytes) ||
+        overlap(k, q_grid, bytes) || overlap(k, k_grid, bytes))
+        return NABLA_ERR_PARAM;
+    if ((st = check_ws(d, NABLA_OP_BUILD_MASK, workspace, workspace_bytes)) != NABLA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
+    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
+    float *qbar = reinterpret_cast<float *>(w);
+    float *kbar_t = reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes);
+    return cuda_status(nabla_launch_build_mask(
+        d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
+        params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
+        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr, s, q_grid,
+        k_grid));
 }
 
 int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
@@ -336,5 +379,5 @@ extern "C" int nabla_build_mask_static(const nabla_shape *shape, const nabla_par
         d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
         params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
         mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr,
-        reinterpret_cast<cudaStream_t>(stream)));
+        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr));
 }

@@ -97,6 +97,89 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restri
 }
 
 // ---------------------------------------------------------------------------
+// fused flatten + pooling: reads Q or K in GRID order [B*h, T, H, W, D], writes
+// the flattened copy [B*h, N, D] and the pooled block means in one pass.
+// Block i is the P x P patch (t, py, px); its flattened token r = yy*P + xx is
+// grid token (t, py*P + yy, px*P + xx).  The means are summed per feature over
+// r ascending exactly as pool_kernel does over the flattened copy, so both
+// paths give the same bits.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) flatten_pool_kernel(
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+    __nv_bfloat16 *__restrict__ qf, __nv_bfloat16 *__restrict__ kf, float *__restrict__ qbar,
+    float *__restrict__ kbar_t, int64_t BH, int nb, int H, int W) {
+    constexpr int CH = D / 8;
+    constexpr int BPC = 256 / CH;  // blocks per CTA
+    constexpr int P = 8;
+    __shared__ float tile[BPC][D + 1];
+    const int tid = threadIdx.x;
+    const int c = tid % CH;
+    const int bl = tid / CH;
+    const int tiles_per_head = (nb + BPC - 1) / BPC;
+    const int64_t cta = blockIdx.x;
+    const int which = static_cast<int>(cta / (BH * tiles_per_head));  // 0: q, 1: k
+    const int64_t rem = cta % (BH * tiles_per_head);
+    const int64_t bh = rem / tiles_per_head;
+    const int i0 = static_cast<int>(rem % tiles_per_head) * BPC;
+    const int i = i0 + bl;
+    const __nv_bfloat16 *x = which ? k : q;
+    __nv_bfloat16 *xf = which ? kf : qf;
+    const int64_t N = static_cast<int64_t>(nb) * kBlk;
+    const int Wp = W / P, HWp = (H / P) * Wp;
+    const int nbp = (nb + 3) & ~3;
+
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    if (i < nb) {
+        const int t = i / HWp, py = (i % HWp) / Wp, px = i % Wp;
+        // grid token of (yy, xx) = first + yy * W + xx
+        const int64_t first = bh * N + (static_cast<int64_t>(t) * H + py * P) * W + px * P;
+        const int4 *src = reinterpret_cast<const int4 *>(x) + c;
+        int4 *dst = reinterpret_cast<int4 *>(xf + (bh * N + static_cast<int64_t>(i) * kBlk) * D) + c;
+#pragma unroll 1
+        for (int r0 = 0; r0 < kBlk; r0 += 16) {
+            int4 v[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int rr = r0 + r;
+                v[r] = __ldg(src + (first + (rr / P) * W + rr % P) * CH);
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                __stcs(dst + (r0 + r) * CH, v[r]);
+                const __nv_bfloat162 *hv = reinterpret_cast<const __nv_bfloat162 *>(&v[r]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float2 f = __bfloat1622float2(hv[e]);
+                    acc[2 * e] = __fadd_rn(acc[2 * e], f.x);
+                    acc[2 * e + 1] = __fadd_rn(acc[2 * e + 1], f.y);
+                }
+            }
+        }
+    }
+    const float inv = 1.0f / kBlk;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = __fmul_rn(acc[e], inv);
+    if (which == 0) {
+        if (i < nb) {
+            float4 *dst = reinterpret_cast<float4 *>(qbar + (bh * nb + i) * D + c * 8);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) tile[bl][c * 8 + e] = acc[e];
+        __syncthreads();
+        for (int idx = tid; idx < D * BPC; idx += 256) {
+            const int d = idx / BPC, b = idx % BPC;
+            if (i0 + b < nb) kbar_t[(bh * D + d) * nbp + i0 + b] = tile[b][d];
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // scores + CDF cut + STA + lists
 // ---------------------------------------------------------------------------
 constexpr int kRows = 16;    // query blocks per CTA
@@ -128,6 +211,32 @@ __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// (frame, patch row, patch column) of block j, advanced by a fixed stride
+// without integer division (the emit loops visit j = lane, lane + 32, ...).
+struct BlockCoord {
+    int t, h, w;
+    __device__ __forceinline__ BlockCoord(int j, int Hp, int Wp)
+        : t(j / (Hp * Wp)), h((j / Wp) % Hp), w(j % Wp) {}
+    __device__ __forceinline__ void advance(int by, int Hp, int Wp) {
+        w += by;
+        while (w >= Wp) {
+            w -= Wp;
+            if (++h == Hp) {
+                h = 0;
+                ++t;
+            }
+        }
+    }
+};
+
+// STA window (section 手法: NABLA, "STA とのハイブリッド統合") in block coordinates:
+// |dt| <= wt/2, |dh| <= wh/2, |dw| <= ww/2.
+__device__ __forceinline__ bool in_window(const BlockCoord &a, const BlockCoord &b,
+                                          const CutParams &prm) {
+    return abs(a.t - b.t) <= prm.wt / 2 && abs(a.h - b.h) <= prm.wh / 2 &&
+           abs(a.w - b.w) <= prm.ww / 2;
 }
 
 // One warp per query row.  E = elements per lane (nb <= 32 * E).
@@ -295,10 +404,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             cstar = (static_cast<uint64_t>(tau) << 16) | xs;
         }
         // emit: bit row + ascending list
-        const int ti = i / (prm.Hp * prm.Wp), hi = (i / prm.Wp) % prm.Hp, wi = i % prm.Wp;
+        const BlockCoord ci(i, prm.Hp, prm.Wp);
+        BlockCoord cj(lane, prm.Hp, prm.Wp);
         int cnt = 0;
         uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
-        for (int w = 0; w < words; ++w) {
+        for (int w = 0; w < words; ++w, cj.advance(32, prm.Hp, prm.Wp)) {
             const int j = w * 32 + lane;
             bool m = false;
             if (j < nb) {
@@ -310,12 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = key >= cstar;
                 }
                 m = m || (j == i) || (prm.flags & 2u);
-                if (!m && !(prm.flags & 1u)) {
-                    const int tj = j / (prm.Hp * prm.Wp), hj = (j / prm.Wp) % prm.Hp,
-                              wj = j % prm.Wp;
-                    m = abs(ti - tj) <= prm.wt / 2 && abs(hi - hj) <= prm.wh / 2 &&
-                        abs(wi - wj) <= prm.ww / 2;
-                }
+                if (!m && !(prm.flags & 1u)) m = in_window(ci, cj, prm);
             }
             const unsigned ball = __ballot_sync(0xffffffffu, m);
             if (lane == 0) bits[(bh * nb + i) * words + w] = ball;
@@ -324,6 +429,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (lane == 0) row_cnt[bh * nb + i] = cnt;
     }
+}
+
+// ---------------------------------------------------------------------------
+// masks that do not depend on the scores: p >= 1 or FULL_STA keeps every
+// block; p <= 0 keeps the STA window and the diagonal (the diagonal alone with
+// NO_STA).  Neither pooling nor scores are needed: one warp per row emits the
+// bit row and the list directly.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) sta_emit_kernel(CutParams prm, int64_t rows,
+                                                      uint32_t *__restrict__ bits,
+                                                      uint16_t *__restrict__ row_idx,
+                                                      int32_t *__restrict__ row_cnt) {
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (r >= rows) return;  // whole warps: rows is per warp
+    const int nb = prm.nb;
+    const int words = (nb + 31) >> 5;
+    const int i = static_cast<int>(r % nb);
+    const bool all = prm.p >= 1.0f || (prm.flags & 2u);
+    const BlockCoord ci(i, prm.Hp, prm.Wp);
+    BlockCoord cj(lane, prm.Hp, prm.Wp);
+    uint16_t *lst = row_idx + r * static_cast<int64_t>(nb);
+    int cnt = 0;
+    for (int w = 0; w < words; ++w, cj.advance(32, prm.Hp, prm.Wp)) {
+        const int j = w * 32 + lane;
+        bool m = false;
+        if (j < nb) m = all || j == i || (!(prm.flags & 1u) && in_window(ci, cj, prm));
+        const unsigned ball = __ballot_sync(0xffffffffu, m);
+        if (lane == 0) bits[r * words + w] = ball;
+        if (m) lst[cnt + __popc(ball & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+        cnt += __popc(ball);
+    }
+    if (lane == 0) row_cnt[r] = cnt;
 }
 
 // ---------------------------------------------------------------------------
@@ -401,34 +539,70 @@ static cudaError_t dispatch_score_cut(dim3 grid, size_t smem, const float *qbar,
     return cudaErrorInvalidValue;
 }
 
+// q_grid/k_grid non-null: q and k are in grid order; flatten them into q/k
+// (then outputs) in the same pass as the pooling.
 cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, float p,
                                     float scale, int wt, int wh, int ww, unsigned flags,
                                     const void *q, const void *k, float *qbar, float *kbar_t,
                                     uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
-                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream) {
+                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream,
+                                    const void *q_grid, const void *k_grid) {
     using namespace nabla;
+    CutParams prm{nb, Hp, Wp, wt, wh, ww, flags, p, scale};
+    cudaError_t err;
+    const bool from_grid = q_grid != nullptr;
     const int bpc = 256 / (D / 8);
     const int64_t tiles = (nb + bpc - 1) / bpc;
     const dim3 pool_grid(static_cast<unsigned>(2 * BH * tiles));
-    if (D == 128)
-        pool_kernel<128><<<pool_grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
-            kbar_t, BH, nb);
-    else
-        pool_kernel<64><<<pool_grid, 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
-            kbar_t, BH, nb);
-    cudaError_t err = cudaGetLastError();
-    if (err != cudaSuccess) return err;
+    if (from_grid) {
+        // flatten (and pool) first: the flattened copies are outputs either way
+        const auto qg = static_cast<const __nv_bfloat16 *>(q_grid);
+        const auto kg = static_cast<const __nv_bfloat16 *>(k_grid);
+        auto qf = static_cast<__nv_bfloat16 *>(const_cast<void *>(q));
+        auto kf = static_cast<__nv_bfloat16 *>(const_cast<void *>(k));
+        if (D == 128)
+            flatten_pool_kernel<128><<<pool_grid, 256, 0, stream>>>(qg, kg, qf, kf, qbar, kbar_t,
+                                                                   BH, nb, Hp * 8, Wp * 8);
+        else
+            flatten_pool_kernel<64><<<pool_grid, 256, 0, stream>>>(qg, kg, qf, kf, qbar, kbar_t,
+                                                                  BH, nb, Hp * 8, Wp * 8);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    if (p <= 0.0f || p >= 1.0f || (flags & 2u)) {
+        // the mask does not depend on the scores
+        const int64_t rows = BH * nb;
+        sta_emit_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
+            prm, rows, bits, row_idx, row_cnt);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+        if (col_idx) {
+            const int64_t warps = BH * ((nb + 31) / 32);
+            col_lists_kernel<<<static_cast<unsigned>((warps + 7) / 8), 256, 0, stream>>>(
+                bits, col_idx, col_cnt, BH, nb);
+            err = cudaGetLastError();
+        }
+        return err;
+    }
+    if (!from_grid) {
+        if (D == 128)
+            pool_kernel<128><<<pool_grid, 256, 0, stream>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
+                kbar_t, BH, nb);
+        else
+            pool_kernel<64><<<pool_grid, 256, 0, stream>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
+                kbar_t, BH, nb);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
 
-    CutParams prm{nb, Hp, Wp, wt, wh, ww, flags, p, scale};
     const size_t smem = nabla_score_cut_smem(nb, D);
     const dim3 grid(static_cast<unsigned>(BH * ((nb + kRows - 1) / kRows)));
     err = D == 128 ? dispatch_score_cut<128>(grid, smem, qbar, kbar_t, prm, bits, row_idx, row_cnt,
                                              stream)
                    : dispatch_score_cut<64>(grid, smem, qbar, kbar_t, prm, bits, row_idx, row_cnt,
                                             stream);
-    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (col_idx) {
         const int64_t warps = BH * ((nb + 31) / 32);

@@ -21,8 +21,8 @@ MASK_BITS, MASK_ROW_IDX, MASK_ROW_CNT, MASK_COL_IDX, MASK_COL_CNT = 0, 1, 2, 3, 
 
 # every symbol include/nabla.h declares
 SYMBOLS = ("nabla_flatten", "nabla_workspace_size", "nabla_mask_bytes", "nabla_build_mask",
-           "nabla_build_mask_static", "nabla_attn_fwd", "nabla_attn_bwd", "nabla_status",
-           "nabla_strerror")
+           "nabla_build_mask_grid", "nabla_build_mask_static", "nabla_attn_fwd", "nabla_attn_bwd",
+           "nabla_status", "nabla_strerror")
 
 
 class NablaError(RuntimeError):
@@ -64,6 +64,8 @@ def lib():
         L.nabla_mask_bytes.restype = SZ
         L.nabla_build_mask.argtypes = [P, P, P, P, P, P, SZ, P]
         L.nabla_build_mask.restype = I
+        L.nabla_build_mask_grid.argtypes = [P, P, P, P, P, P, P, P, SZ, P]
+        L.nabla_build_mask_grid.restype = I
         L.nabla_build_mask_static.argtypes = [P, P, P, P, P, P]
         L.nabla_build_mask_static.restype = I
         L.nabla_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, P, SZ, P]
@@ -172,6 +174,23 @@ def build_mask(shape, params, q, k, mask=None, ws=None):
                                   ctypes.byref(ms), _ptr(ws), ws.numel(), _stream(q)),
            "nabla_build_mask")
     return mask
+
+
+def build_mask_grid(shape, params, q_grid, k_grid, q=None, k=None, mask=None, ws=None):
+    """Flatten q_grid, k_grid (grid order, any shape holding [B*h, T*H*W, D])
+    into q, k and build the mask from them in one call; returns (q, k, mask)."""
+    _need(q_grid, torch.bfloat16, "q_grid")
+    _need(k_grid, torch.bfloat16, "k_grid")
+    q = torch.empty_like(q_grid) if q is None else q
+    k = torch.empty_like(k_grid) if k is None else k
+    cols = bool(params.flags & EMIT_COLS)
+    mask = alloc_mask(shape, q_grid.device, cols) if mask is None else mask
+    ws = workspace(shape, OP_BUILD_MASK, q_grid.device) if ws is None else ws
+    ms = _mask_struct(mask)
+    _check(lib().nabla_build_mask_grid(ctypes.byref(shape), ctypes.byref(params), _ptr(q_grid),
+                                       _ptr(k_grid), _ptr(q), _ptr(k), ctypes.byref(ms), _ptr(ws),
+                                       ws.numel(), _stream(q_grid)), "nabla_build_mask_grid")
+    return q, k, mask
 
 
 def attn_fwd(shape, params, q, k, v, mask, o=None, lse=None, ws=None, want_lse=True):

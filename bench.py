@@ -256,11 +256,11 @@ def run_nabla(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(src, ev=None):
-        for n in ("q", "k", "v"):
-            nabla.flatten(src[n], w.T, w.H, w.W, w.P, out=B["flat"][n])
+        nabla.flatten(src["v"], w.T, w.H, w.W, w.P, out=B["flat"]["v"])
         if ev: ev[1].record(stream)
-        nabla.build_mask(shape, prm, B["flat"]["q"], B["flat"]["k"], mask=B["mask"],
-                         ws=B["ws_mask"])
+        # Q and K are flattened by the mask build itself (pooling in the same pass)
+        nabla.build_mask_grid(shape, prm, src["q"], src["k"], q=B["flat"]["q"], k=B["flat"]["k"],
+                              mask=B["mask"], ws=B["ws_mask"])
         if ev: ev[2].record(stream)
         nabla.attn_fwd(shape, prm, B["flat"]["q"], B["flat"]["k"], B["flat"]["v"], B["mask"],
                        o=B["o"], lse=B["lse"], ws=B["ws_fwd"])
@@ -272,7 +272,7 @@ def run_nabla(args):
         for n in ("o", "dq", "dk", "dv"):
             nabla.flatten(B[n], w.T, w.H, w.W, w.P, inverse=True, out=B["out"][n])
 
-    launches_per_step = 3 + 3 + 1 + 3 + 4  # flatten, pool/score_cut/cols, fwd, bwd x3, unflatten
+    launches_per_step = 1 + 3 + 1 + 3 + 4  # flatten v, flatten_pool/score_cut/cols, fwd, bwd x3, unflatten
 
     def barrier():
         if world > 1:
@@ -318,10 +318,12 @@ def run_nabla(args):
     bwd_flop = 10.0 * 64 * 64 * w.D * kept
     value = world * (fwd_flop + bwd_flop) / (ms_step * 1e-3) / 1e12
     N, D, BH, nb = w.N, w.D, w.BH, w.nb
-    mask_bytes = (4.0 * N * D * BH + 16.0 * nb * D * BH + nb * nb * BH / 8.0
+    # flatten of Q and K (read grid, write flattened) + pooled means (write + read)
+    # + bit rows + row and column lists
+    mask_bytes = (2 * 4.0 * N * D * BH + 16.0 * nb * D * BH + nb * nb * BH / 8.0
                   + 2 * 2.0 * kept + 2 * 4.0 * BH * nb)
     mask_gbs = mask_bytes / (phase[1] * 1e-3) / 1e9
-    flat_gbs = 3 * 2.0 * BH * N * D * 2 / (phase[0] * 1e-3) / 1e9
+    flat_gbs = 2.0 * BH * N * D * 2 / (phase[0] * 1e-3) / 1e9
 
     pk, pk_src = peaks()
     ops = {"attn_bwd": (phase[3], bwd_flop), "attn_fwd": (phase[2], fwd_flop)}
@@ -385,14 +387,15 @@ def run_nabla(args):
             "data": "synthetic: seeded cell-correlated bf16 Q/K/V (cell 2x8x8, noise 0.5), dO ~ "
                     "N(0,1); each rank its own batch",
             "config": workload_config(w),
-            "breakdown_ms": {"flatten_qkv": phase[0], "build_mask": phase[1],
+            "breakdown_ms": {"flatten_v": phase[0], "flatten_qk_build_mask": phase[1],
                              "attn_fwd": phase[2], "attn_bwd": phase[3],
                              "unflatten_out": phase[4]},
             "kept_blocks": kept, "kept_fraction": kept_frac,
             "attn_fwd_tflops": fwd_flop / (phase[2] * 1e-3) / 1e12,
             "attn_bwd_tflops": bwd_flop / (phase[3] * 1e-3) / 1e12,
-            "mask_build_gbs": mask_gbs, "mask_build_frac_hbm": mask_gbs / pk["hbm_gbs"],
-            "flatten_gbs": flat_gbs,
+            "flatten_qk_build_mask_gbs": mask_gbs,
+            "flatten_qk_build_mask_frac_hbm": mask_gbs / pk["hbm_gbs"],
+            "flatten_v_gbs": flat_gbs,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": launches_per_step * args.steps,
         }

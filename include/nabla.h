@@ -145,11 +145,32 @@ size_t nabla_mask_bytes(const nabla_shape *shape, int part);
  *                    summed u reaches p * sum_j u_ij (float64 product);
  *   M_ij           = adaptive OR STA window OR (i == j).
  * Writes bits, row lists, and (with NABLA_EMIT_COLS) column lists.
+ * When M does not depend on the scores -- p >= 1 or NABLA_FULL_STA (every
+ * block), p <= 0 (STA window and diagonal; the diagonal alone with
+ * NABLA_NO_STA) -- q and k are not read and no pooling or scores are computed
+ * (the pure-STA configuration runs at list-emission cost); the arguments are
+ * validated as usual.
  * Workspace: nabla_workspace_size(shape, NABLA_OP_BUILD_MASK) bytes, 256-byte
  * aligned. */
 int nabla_build_mask(const nabla_shape *shape, const nabla_params *params,
                      const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
                      void *workspace, size_t workspace_bytes, nabla_stream_t stream);
+
+/* Flattening of Q and K fused with the mask build (sections 手法: NABLA,
+ * "トークン再順序付け (Fractal Flattening)" and "適応型マスク構築"): the
+ * same outputs as nabla_flatten(q_grid -> q), nabla_flatten(k_grid -> k)
+ * followed by nabla_build_mask(q, k), with the pooling done in the flattening
+ * pass instead of re-reading the flattened copies.
+ *   q_grid, k_grid  [B, heads, T, H, W, D] bf16 in grid order (inputs);
+ *   q, k            [B, heads, N, D] bf16, written in flattened order (outputs;
+ *                   the attention calls take them);
+ *   mask, workspace as nabla_build_mask; the pooled means are bit-identical.
+ * q and k must not overlap each other or either input (NABLA_ERR_PARAM).  All
+ * four pointers 16-byte aligned.  Other checks as nabla_build_mask. */
+int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
+                          const nabla_bf16 *q_grid, const nabla_bf16 *k_grid, nabla_bf16 *q,
+                          nabla_bf16 *k, const nabla_mask *mask, void *workspace,
+                          size_t workspace_bytes, nabla_stream_t stream);
 
 /* Same computation and outputs as nabla_build_mask, without a workspace.
  * (No counterpart on the page: this is a calling convenience.)

@@ -100,6 +100,26 @@ def test_build_mask_rejects_on_host(L):
                               1 << 40, None) == nabla.ERR_NULL
 
 
+def test_build_mask_grid_rejects_on_host(L):
+    s, good = _shape(), nabla.params_of(0.7, (3, 3, 3), D=128)
+    bytes_ = 2 * s.B * s.heads * s.T * s.H * s.W * s.D
+    a, b = ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000 + bytes_)
+    c, d = ctypes.c_void_p(0x10000 + 2 * bytes_), ctypes.c_void_p(0x10000 + 3 * bytes_)
+
+    def g(qg, kg, q, k, mask=None, params=good, ws_bytes=1 << 40):
+        m = _mask() if mask is None else mask
+        return L.nabla_build_mask_grid(ctypes.byref(s), ctypes.byref(params), qg, kg, q, k,
+                                       ctypes.byref(m), FAKE, ws_bytes, None)
+    assert g(None, b, c, d) == nabla.ERR_NULL
+    assert g(a, b, c, None) == nabla.ERR_NULL
+    assert g(a, b, FAKE_ODD, d) == nabla.ERR_ALIGN
+    assert g(a, b, c, c) == nabla.ERR_PARAM                                  # q overlaps k
+    assert g(a, b, a, d) == nabla.ERR_PARAM                                  # in place
+    assert g(a, b, ctypes.c_void_p(0x10000 + bytes_ // 2), d) == nabla.ERR_PARAM  # partial overlap
+    assert g(a, b, c, d, ws_bytes=1024) == nabla.ERR_WORKSPACE
+    assert g(a, b, c, d, params=nabla.params_of(1.5, (3, 3, 3), D=128)) == nabla.ERR_PARAM
+
+
 def test_attention_rejects_on_host(L):
     s, good = _shape(), nabla.params_of(0.7, (3, 3, 3), D=128)
     m = _mask()

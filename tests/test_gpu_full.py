@@ -120,3 +120,40 @@ def test_long_forward_sampled(long92, p, heads, blocks):
     oo, _ = oracle.attn_fwd(x["q"], x["k"], x["v"], sm["row_idx"], sm["row_cnt"], w.scale, sel=sel)
     go = o.view(w.BH, w.nb, L, w.D)
     assert_close(np.stack([bf16_to_f64(go[heads[hh], i]) for hh, i in sel]), oo, "O")
+
+
+@pytest.fixture(scope="module")
+def max2048():
+    # the largest block count the library accepts: T=32, 64x64 latent -> 32 x 8 x 8 = 2048
+    # blocks of 64 tokens (131,072 tokens), one head, with a training backward
+    return Case(synth.Workload("max2048", 1, 1, 32, 64, 64, 128, (2, 8, 8), 0.7, backward=True))
+
+
+def test_max_blocks_mask_every_row(max2048):
+    assert max2048.w.nb == 2048
+    gm = to_np(max2048.gpu_mask())
+    om = max2048.oracle_mask()
+    assert check_mask(gm, om) == 0
+
+
+def test_max_blocks_forward_and_backward_sampled(max2048):
+    c, w = max2048, max2048.w
+    om = c.oracle_mask()
+    gm = c.gpu_mask()
+    o, lse = _sampled_forward(c, om, gm, heads=(0,), blocks_per_head=12, seed=4)
+    dq, dk, dv = nabla.attn_bwd(c.shape, c.params(), c.gpu["q"], c.gpu["k"], c.gpu["v"], o,
+                                c.gpu["dout"], lse, gm)
+    torch.cuda.synchronize()
+    x = _heads_f64(c, ("q", "k", "v", "dout"), (0,))
+    rng = np.random.default_rng(5)
+    dq_sel = [(0, int(i)) for i in rng.choice(w.nb, 6, replace=False)]
+    kv_sel = [(0, 0), (0, w.nb - 1)]  # the first and the last key block
+    oq, ok_, ov = oracle.attn_bwd(x["q"], x["k"], x["v"], x["dout"], om["row_idx"], om["row_cnt"],
+                                  om["col_idx"], om["col_cnt"], w.scale, dq_sel=dq_sel,
+                                  kv_sel=kv_sel)
+    gq = dq.view(w.BH, w.nb, L, w.D)
+    gk = dk.view(w.BH, w.nb, L, w.D)
+    gv = dv.view(w.BH, w.nb, L, w.D)
+    assert_close(np.stack([bf16_to_f64(gq[0, i]) for _, i in dq_sel]), oq, "dQ")
+    assert_close(np.stack([bf16_to_f64(gk[0, j]) for _, j in kv_sel]), ok_, "dK")
+    assert_close(np.stack([bf16_to_f64(gv[0, j]) for _, j in kv_sel]), ov, "dV")

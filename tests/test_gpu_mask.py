@@ -74,3 +74,64 @@ def test_deterministic(small):
     b = to_np(small.gpu_mask())
     for k in a:
         assert np.array_equal(a[k], b[k]), k
+
+
+# Masks that do not depend on the scores (p <= 0, p >= 1, FULL_STA) take a
+# path with neither pooling nor scores; windows other than 3x3x3 and patch
+# grids narrower and wider than a warp exercise its block-coordinate stepping.
+SCORE_FREE = [
+    synth.Workload("win531_w5", 1, 2, 6, 24, 40, 64, (1, 4, 4), 0.7, window=(5, 3, 1)),     # Wp = 5
+    synth.Workload("win173_w40", 1, 1, 3, 16, 320, 64, (1, 4, 4), 0.7, window=(1, 7, 3)),   # Wp = 40
+    synth.Workload("win999", 1, 1, 4, 32, 32, 128, (2, 4, 4), 0.7, window=(9, 9, 9)),       # window > grid
+]
+
+
+@pytest.mark.parametrize("w", SCORE_FREE, ids=lambda w: w.name)
+@pytest.mark.parametrize("p,flags", [(0.0, 0), (0.0, nabla.NO_STA), (1.0, 0), (0.5, nabla.FULL_STA),
+                                     (0.6, 0)])
+def test_score_free_paths_and_windows(w, p, flags):
+    c = Case(w)
+    gm = to_np(c.gpu_mask(p, flags))
+    om = c.oracle_mask(p, flags)
+    assert check_mask(gm, om) == 0
+    if p >= 1.0 or flags & nabla.FULL_STA:
+        assert np.all(gm["row_cnt"] == w.nb)
+    if p == 0.0 and flags & nabla.NO_STA:
+        assert np.all(gm["row_cnt"] == 1)  # the diagonal alone
+
+
+GRID = [synth.WORKLOADS["small"], ODD[1], ODD[3], SCORE_FREE[1]]
+
+
+@pytest.mark.parametrize("w", GRID, ids=lambda w: w.name)
+@pytest.mark.parametrize("p,flags", [(None, 0), (0.0, 0), (0.5, nabla.FULL_STA)])
+def test_build_mask_from_grid_matches_flatten_then_build(w, p, flags):
+    """nabla_build_mask_grid: flattened copies bit-identical to the oracle's
+    flattening, pooled means bit-identical to the oracle's pooling, and the
+    mask identical to the one built from the separately flattened tensors."""
+    c = Case(w)
+    inp = synth.make_inputs(w, 0, with_dout=False)
+    qg = inp["q"].reshape(w.BH, w.N, w.D).cuda()
+    kg = inp["k"].reshape(w.BH, w.N, w.D).cuda()
+    prm = c.params(p, flags)
+    ws = nabla.workspace(c.shape, nabla.OP_BUILD_MASK, "cuda")
+    qf, kf, gm = nabla.build_mask_grid(c.shape, prm, qg, kg, ws=ws)
+    torch.cuda.synchronize()
+    assert nabla.status(ws) == nabla.OK
+    assert np.array_equal(synth.bits(qf.cpu()), c.cpu["q"])
+    assert np.array_equal(synth.bits(kf.cpu()), c.cpu["k"])
+    ref = to_np(c.gpu_mask(p, flags))
+    got = to_np(gm)
+    for key in ref:
+        if key in ("row_idx", "col_idx"):
+            cnt = ref["row_cnt" if key == "row_idx" else "col_cnt"]
+            valid = np.arange(w.nb)[None, None, :] < cnt[..., None]
+            assert np.array_equal(np.where(valid, got[key], 0), np.where(valid, ref[key], 0)), key
+        else:
+            assert np.array_equal(got[key], ref[key]), key
+    assert check_mask(got, c.oracle_mask(p, flags)) == 0
+    if p is None:  # the scored path pooled from the grid layout
+        n = w.BH * w.nb * w.D
+        raw = ws.cpu().numpy()
+        qbar = raw[256:256 + 4 * n].view(np.float32).reshape(w.BH, w.nb, w.D)
+        assert np.array_equal(qbar, oracle.pool_f32(c.cpu["q"]))
