@@ -46,7 +46,7 @@ NCU_DRAM_BYTES_PER_HEAD = {
 }
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
@@ -59,7 +59,7 @@ def parse():
                     help="train: 720p-like training step (the benchmark); long: 92,160-token clip")
     ap.add_argument("--heads", type=int, default=None,
                     help="run fewer heads (profiling captures only; not a benchmark result)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def workload_of(args):
@@ -196,6 +196,22 @@ def dist_init(n):
     return rank, world, local
 
 
+def max_over_ranks(x, world, device):
+    """Maximum of a per-rank scalar over all ranks (every rank gets it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(flop_per_rank, ms_per_step, world):
+    """Weak scaling: every rank runs the whole workload on its own batch, so
+    the job processes world x the per-rank FLOPs in the slowest rank's time."""
+    return world * flop_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def run_reference(args):
     rank, world, _ = dist_init(args.gpus)
     if rank != 0:
@@ -280,11 +296,6 @@ def run_nabla(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    def max_over_ranks(x):
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(args.warmup):
         step(grid)
@@ -307,7 +318,7 @@ def run_nabla(args):
     stop.record(stream)
     barrier()
     clk = clocks.stop()
-    total_ms = max_over_ranks(start.elapsed_time(stop))
+    total_ms = max_over_ranks(start.elapsed_time(stop), world, dev)
     phase = [0.0] * 5
     for s in range(args.steps):
         for p in range(5):
@@ -317,7 +328,7 @@ def run_nabla(args):
 
     fwd_flop = 4.0 * 64 * 64 * w.D * kept
     bwd_flop = 10.0 * 64 * 64 * w.D * kept
-    value = world * (fwd_flop + bwd_flop) / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(fwd_flop + bwd_flop, ms_step, world)
     N, D, BH, nb = w.N, w.D, w.BH, w.nb
     # flatten of Q and K (read grid, write flattened) + pooled means (write + read)
     # + bit rows + row and column lists
@@ -403,10 +414,10 @@ def run_nabla(args):
         run(args.steps)
         b_.record(stream)
         barrier()
-        e2e_ms = max_over_ranks(a.elapsed_time(b_)) / args.steps
+        e2e_ms = max_over_ranks(a.elapsed_time(b_), world, dev) / args.steps
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-        e2e = {"value": world * (fwd_flop + bwd_flop) / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": whole_job_tflops(fwd_flop + bwd_flop, e2e_ms, world), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "copies": "pinned host <-> device on a copy stream, overlapped with the "
                          "neighbouring steps' compute"}
