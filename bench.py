@@ -55,6 +55,8 @@ def parse(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the long-clip p sweep (kept fraction vs time) added to the line")
     ap.add_argument("--workload", default=WORKLOAD, choices=("train", "long"),
                     help="train: 720p-like training step (the benchmark); long: 92,160-token clip")
     ap.add_argument("--heads", type=int, default=None,
@@ -210,6 +212,53 @@ def whole_job_tflops(flop_per_rank, ms_per_step, world):
     """Weak scaling: every rank runs the whole workload on its own batch, so
     the job processes world x the per-rank FLOPs in the slowest rank's time."""
     return world * flop_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
+def long_p_sweep(dev, reps=5, warmup=3):
+    """Kept-block fraction against time on the long clip (92,160 tokens,
+    12 heads, 1,440 blocks) for each p of its sweep: mask build from the
+    flattened Q, K and the block-sparse forward, each timed with CUDA events
+    (median of `reps` after `warmup`)."""
+    import statistics as st
+    import torch
+    from adaptive_block_sparse_fractal_b200 import nabla, synth
+    w = synth.WORKLOADS["long"]
+    shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
+    grid = synth.make_inputs_device(w, 0, dev, with_dout=False)
+    q, k, v = (nabla.flatten(grid[n], w.T, w.H, w.W, w.P) for n in ("q", "k", "v"))
+    del grid
+    stream = torch.cuda.current_stream(dev)
+    mask = nabla.alloc_mask(shape, dev, cols=False)
+    ws_m = nabla.workspace(shape, nabla.OP_BUILD_MASK, dev)
+    ws_f = nabla.workspace(shape, nabla.OP_ATTN_FWD, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.BH, w.N), dtype=torch.float32, device=dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        out = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            out.append(a.elapsed_time(b))
+        return st.median(out)
+
+    rows = []
+    for p in w.p_sweep:
+        prm = nabla.params_of(p, w.window, D=w.D)
+        t_mask = timed(lambda: nabla.build_mask(shape, prm, q, k, mask=mask, ws=ws_m))
+        t_fwd = timed(lambda: nabla.attn_fwd(shape, prm, q, k, v, mask, o=o, lse=lse, ws=ws_f))
+        kept = int(mask["row_cnt"].sum().item())
+        rows.append({"p": p, "kept_fraction": kept / (w.BH * w.nb * w.nb),
+                     "build_mask_ms": t_mask, "attn_fwd_ms": t_fwd,
+                     "attn_fwd_tflops": 4.0 * 64 * 64 * w.D * kept / (t_fwd * 1e-3) / 1e12})
+    return {"workload": "long: B=1 heads=12 T*H*W=60x32x48 (92160 tokens, 1440 blocks) D=128 "
+                        "STA 3x3x3, cell 2x4x4; mask from flattened Q,K + forward per p",
+            "rows": rows}
 
 
 def run_reference(args):
@@ -423,6 +472,12 @@ def run_nabla(args):
                          "neighbouring steps' compute"}
         del dev_in, dev_out
 
+    sweep = None
+    if rank == 0 and world == 1 and not args.no_sweep:
+        B.clear()  # free this workload's buffers first
+        torch.cuda.empty_cache()
+        sweep = long_p_sweep(dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         flop, t_fwd, t_mask, cores, desc = oracle_sample(w)
@@ -447,6 +502,7 @@ def run_nabla(args):
             "flatten_qk_build_mask_frac_hbm": mask_gbs / pk["hbm_gbs"],
             "flatten_v_gbs": flat_gbs,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "long_p_sweep": sweep,
             "gpu_launches": launches_per_step * args.steps,
         }
         print(json.dumps(line), flush=True)
