@@ -31,7 +31,7 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
                                         const uint16_t *row_idx, const int32_t *row_cnt,
                                         const uint16_t *col_idx, const int32_t *col_cnt,
                                         void *dq, void *dk, void *dv, float *dl, float *l2,
-                                        int *status, cudaStream_t stream);
+                                        int *status, int force_timeout, cudaStream_t stream);
 cudaError_t nabla_launch_attn_bwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
                                       const void *k, const void *v, const void *o,
                                       const void *dout, const float *lse, const uint16_t *row_idx,
@@ -286,7 +286,7 @@ int nabla_attn_bwd(const nabla_shape *shape, const nabla_params *params, const n
         return cuda_status(nabla_launch_attn_bwd_sm100(
             d.BH, d.nb, d.Hp, d.Wp, shape->T, params->scale, q, k, v, o, dout, lse, mask->row_idx,
             mask->row_cnt, mask->col_idx, mask->col_cnt, dq, dk, dv, dl, l2,
-            static_cast<int *>(workspace), s));
+            static_cast<int *>(workspace), (params->flags & NABLA_DEBUG_TIMEOUT) ? 1 : 0, s));
     }
     return cuda_status(nabla_launch_attn_bwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v, o,
                                                  dout, lse, mask->row_idx, mask->row_cnt,

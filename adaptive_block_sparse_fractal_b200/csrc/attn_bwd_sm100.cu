@@ -76,7 +76,7 @@ constexpr uint32_t KV_U = KV_RING + kStages * kStageBytes;  // union list
 constexpr uint32_t KV_UF = KV_U + 2 * (kMaxNbBwd + 8);
 constexpr uint32_t KV_CB = ((KV_UF + kMaxNbBwd + 8 + 15) / 16) * 16;  // column bits [2][64]
 constexpr uint32_t KV_BAR = KV_CB + 2 * 256;
-constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1;
+constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
 constexpr uint32_t KV_INT = KV_BAR + 8 * kKvBars;
 constexpr uint32_t kKvSmem = KV_INT + 16 + 1024;
 
@@ -91,7 +91,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 const uint16_t *__restrict__ col_idx, const int32_t *__restrict__ col_cnt,
                 __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
                 int *__restrict__ status, int nb, int Hp, int Wp, int T, float c, float scale,
-                uint32_t wait_limit) {
+                uint32_t wait_limit, int force_timeout) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // pd_full[t & 1]: the eight softmax warps wrote P^T(t), dS^T(t) (two
     // barriers, so a warp already on tile t+1 cannot complete tile t's phase)
     uint64_t *s_full = bar + 1 + 2 * kStages, *pd_full = s_full + 2, *done = pd_full + 2;
+    uint64_t *never = done + 1;  // nothing arrives here (timeout test aid)
     int *sInt = reinterpret_cast<int *>(sm + KV_INT);
     volatile int *abort_flag = sInt + 2;
 
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             mbar_init(&pd_full[b], 8);
         }
         mbar_init(done, 1);
+        mbar_init(never, 1);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
     }
@@ -249,6 +251,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const int kh = tw >> 6;          // key block of the pair
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         bool ok = true;
+        if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
         for (int t = 0; t < ntiles; ++t) {
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
@@ -357,7 +360,7 @@ constexpr uint32_t DQ_RB = DQ_RING + kDqRing * kDqSlot;   // row bits [2][64]
 constexpr uint32_t DQ_U = DQ_RB + 2 * 256;                // union list u16
 constexpr uint32_t DQ_UF = DQ_U + 2 * (kMaxNbBwd + 8);    // membership per entry
 constexpr uint32_t DQ_BAR = ((DQ_UF + kMaxNbBwd + 8 + 7) / 8) * 8;
-constexpr int kDqBars = 2 * kDqRing + 2 + 2 + 1 + 1;
+constexpr int kDqBars = 2 * kDqRing + 2 + 2 + 1 + 1 + 1;
 constexpr uint32_t DQ_INT = DQ_BAR + 8 * kDqBars;
 constexpr uint32_t kDqSmem = DQ_INT + 16 + 1024;
 
@@ -367,7 +370,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
               const float *__restrict__ l2, const float *__restrict__ dl,
               const uint16_t *__restrict__ row_idx, const int32_t *__restrict__ row_cnt,
               __nv_bfloat16 *__restrict__ dq, int *__restrict__ status, int nb, int Hp, int Wp,
-              int T, float c, float scale, uint32_t wait_limit) {
+              int T, float c, float scale, uint32_t wait_limit, int force_timeout) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
@@ -381,6 +384,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     // ds_full[t & 1]: the eight dS warps wrote dS(t) (two barriers, so a warp
     // already on tile t+1 cannot complete tile t's phase for the others)
     uint64_t *ds_full = s_full + 2, *q_ready = ds_full + 2, *done = q_ready + 1;
+    uint64_t *never = done + 1;  // nothing arrives here (timeout test aid)
     int *sInt = reinterpret_cast<int *>(sm + DQ_INT);  // [0] tmem base [1] tiles [2] abort
     volatile int *abort_flag = sInt + 2;
 
@@ -406,6 +410,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
         mbar_init(q_ready, 8);
         mbar_init(done, 1);
+        mbar_init(never, 1);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
     }
@@ -512,6 +517,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const int ib = h ? (iB >= 0 ? iB : iA) : iA;
         const int64_t grow = bh * N + static_cast<int64_t>(ib) * kBlk + (r & 63);
         const float Lr = l2[grow], Dr = dl[grow];
+        bool ok = true;
+        if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
         {
             // Q (group 0) or dO (group 1) row -> TMEM, the A operands of S and dP
             const uint4 *src = reinterpret_cast<const uint4 *>((kg ? dout : q) + grow * kD);
@@ -535,7 +542,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(q_ready);
 
-        bool ok = true;
         for (int t = 0; t < ntiles; ++t) {
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
@@ -609,7 +615,7 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
                                         const uint16_t *row_idx, const int32_t *row_cnt,
                                         const uint16_t *col_idx, const int32_t *col_cnt,
                                         void *dq, void *dk, void *dv, float *dl, float *l2,
-                                        int *status, cudaStream_t stream) {
+                                        int *status, int force_timeout, cudaStream_t stream) {
     using namespace nabla::bwd100;
     const int64_t rows = BH * static_cast<int64_t>(nb) * nabla::kBlk;
     if (rows >= (1ll << 31) || nb > kMaxNbBwd) return cudaErrorInvalidValue;
@@ -630,7 +636,7 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
     const int64_t groups = static_cast<int64_t>((T + 1) / 2) * Hp * Wp;
     dkdv_kernel<<<static_cast<unsigned>(BH * groups), kKvThreads, kKvSmem, stream>>>(
         mq, mk, mv, mdo, l2, dl, col_idx, col_cnt, static_cast<__nv_bfloat16 *>(dk),
-        static_cast<__nv_bfloat16 *>(dv), status, nb, Hp, Wp, T, c, scale, limit);
+        static_cast<__nv_bfloat16 *>(dv), status, nb, Hp, Wp, T, c, scale, limit, force_timeout);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     err = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -639,6 +645,6 @@ cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int 
     dq_kernel<<<static_cast<unsigned>(BH * groups), kDqThreads, kDqSmem, stream>>>(
         mk, mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(dout),
         l2, dl, row_idx, row_cnt, static_cast<__nv_bfloat16 *>(dq), status, nb, Hp, Wp, T, c,
-        scale, limit);
+        scale, limit, force_timeout);
     return cudaGetLastError();
 }

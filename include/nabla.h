@@ -56,10 +56,11 @@ typedef struct CUstream_st *nabla_stream_t; /* == cudaStream_t */
 #define NABLA_NO_STA 1u    /* no STA term: M = adaptive OR diagonal            */
 #define NABLA_FULL_STA 2u  /* STA window covers every block: dense attention   */
 #define NABLA_EMIT_COLS 4u /* also write the column lists needed by the backward */
-/* Test aid, not for production: makes the tensor-core attention forward give
- * up its first device-side wait at once, so that the timeout path (status
- * word = NABLA_ERR_TIMEOUT, clean unwind, context still usable) can be
- * exercised without faulting or hanging the GPU.  Outputs are not written. */
+/* Test aid, not for production: makes the tensor-core attention forward and
+ * backward (D = 128) give up a device-side wait at once, so that the timeout
+ * path (status word = NABLA_ERR_TIMEOUT, clean unwind, context still usable)
+ * can be exercised without faulting or hanging the GPU.  Outputs are not
+ * meaningful after it. */
 #define NABLA_DEBUG_TIMEOUT 0x100u
 
 /* Problem shape.  P must be 8. */

@@ -124,6 +124,30 @@ def test_forward_timeout_is_reported_and_the_context_survives():
     assert_close(bf16_to_f64(o).reshape(-1, L, w.D), oo, "O after timeout")
 
 
+def test_backward_timeout_is_reported_and_the_context_survives():
+    # As for the forward: the flag makes the backward's first device-side wait
+    # (in the dK/dV kernel; the dQ kernel then sees the status and skips) give
+    # up at once; the status must read NABLA_ERR_TIMEOUT and the next backward
+    # on the same context and workspace must be correct.
+    w = synth.Workload("odd130b", 1, 2, 5, 16, 104, 128, (2, 4, 4), 0.7, backward=True)
+    c = Case(w)
+    gm = c.gpu_mask()
+    o, lse = nabla.attn_fwd(c.shape, c.params(), c.gpu["q"], c.gpu["k"], c.gpu["v"], gm)
+    ws = nabla.workspace(c.shape, nabla.OP_ATTN_BWD, "cuda")
+    args = (c.gpu["q"], c.gpu["k"], c.gpu["v"], o, c.gpu["dout"], lse, gm)
+    nabla.attn_bwd(c.shape, c.params(flags=nabla.DEBUG_TIMEOUT), *args, ws=ws)
+    assert nabla.status(ws) == nabla.ERR_TIMEOUT
+    dq, dk, dv = nabla.attn_bwd(c.shape, c.params(), *args, ws=ws)
+    assert nabla.status(ws) == nabla.OK
+    om = c.oracle_mask()
+    q, k, v, do = (f64(c.cpu[n]) for n in ("q", "k", "v", "dout"))
+    gq, gk, gv = oracle.attn_bwd(q, k, v, do, om["row_idx"], om["row_cnt"], om["col_idx"],
+                                 om["col_cnt"], w.scale)
+    for name, got, want in (("dQ", dq, gq), ("dK", dk, gk), ("dV", dv, gv)):
+        assert_close(bf16_to_f64(got).reshape(-1, L, w.D), want.reshape(-1, L, w.D),
+                     name + " after timeout")
+
+
 def _extreme_scores(inp):
     # Every query gets a large component along feature 0 and one key per head a
     # large component along feature 1: scores span hundreds of units, so a
