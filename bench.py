@@ -37,12 +37,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, per
-# head, from one ncu --set full capture of `bench.py --heads 8` (same shape,
+# head, from one ncu capture of `bench.py --heads 8 --no-sweep` (same shape,
 # 8 heads; heads are independent, so the traffic scales with their number).
 # Must be re-measured whenever these kernels change.
 NCU_DRAM_BYTES_PER_HEAD = {
-    ("train", "attn_bwd"): (324.7e6 + 956.0e6 + 792.7e6) / 8,  # pre + dK/dV + dQ
-    ("train", "attn_fwd"): (476.3e6 + 146.1e6) / 8,
+    ("train", "attn_bwd"): (320.8e6 + 951.1e6 + 788.5e6) / 8,  # pre + dK/dV + dQ
+    ("train", "attn_fwd"): (475.9e6 + 144.8e6) / 8,
 }
 
 
