@@ -59,8 +59,9 @@ __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restric
 #pragma unroll
     for (int off = 1; off < 16; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (row < rows && sub == 0) {
-        dl[row] = acc;
-        l2[row] = lse[row] * 1.4426950408889634f;
+        // stored negated, the form the packed exponent and difference take
+        dl[row] = -acc;
+        l2[row] = -(lse[row] * 1.4426950408889634f);
     }
 }
 
@@ -271,17 +272,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     const float4 l4 = L4[q4], d4 = D4[q4];
                     const float la[4] = {l4.x, l4.y, l4.z, l4.w};
                     const float da[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pv[4], gv[4];
+                    // la = -L log2(e), da = -D (stored negated): per pair of
+                    // queries P = exp2(s c - L), dS = P (dP - D), packed
+                    const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
+                    for (int e = 0; e < 4; e += 2) {
                         const int q = 4 * q4 + e;
-                        pv[e] = fast_exp2(fmaf(sv[q], c, -la[e]));
-                        gv[e] = pv[e] * (dp[q] - da[e]);
+                        const uint64_t x = f2_fma(f2_pack(sv[q], sv[q + 1]), c2, f2_pack(la[e], la[e + 1]));
+                        const float p0 = fast_exp2(f2_lo(x)), p1 = fast_exp2(f2_hi(x));
+                        const uint64_t g = f2_mul(f2_pack(p0, p1),
+                                                  f2_add(f2_pack(dp[q], dp[q + 1]), f2_pack(da[e], da[e + 1])));
+                        pk[2 * q4 + (e >> 1)] = pack_bf16(p0, p1);
+                        dk2[2 * q4 + (e >> 1)] = pack_bf16(f2_lo(g), f2_hi(g));
                     }
-                    pk[2 * q4] = pack_bf16(pv[0], pv[1]);
-                    pk[2 * q4 + 1] = pack_bf16(pv[2], pv[3]);
-                    dk2[2 * q4] = pack_bf16(gv[0], gv[1]);
-                    dk2[2 * q4 + 1] = pack_bf16(gv[2], gv[3]);
                 }
             } else {
 #pragma unroll
@@ -516,7 +519,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         const int ib = h ? (iB >= 0 ? iB : iA) : iA;
         const int64_t grow = bh * N + static_cast<int64_t>(ib) * kBlk + (r & 63);
-        const float Lr = l2[grow], Dr = dl[grow];
+        const float nLr = l2[grow], nDr = dl[grow];  // -L log2(e), -D
         bool ok = true;
         if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
         {
@@ -553,11 +556,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 tmem_ld32(scol, sv);
                 tmem_ld32(scol + 64, dp);
                 tmem_wait_ld();
+                const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(nLr, nLr), nd2 = f2_pack(nDr, nDr);
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
-                    const float p0 = fast_exp2(fmaf(sv[e], c, -Lr));
-                    const float p1 = fast_exp2(fmaf(sv[e + 1], c, -Lr));
-                    gk[e >> 1] = pack_bf16(p0 * (dp[e] - Dr), p1 * (dp[e + 1] - Dr));
+                    const uint64_t x = f2_fma(f2_pack(sv[e], sv[e + 1]), c2, nl2);
+                    const uint64_t g = f2_mul(f2_pack(fast_exp2(f2_lo(x)), fast_exp2(f2_hi(x))),
+                                              f2_add(f2_pack(dp[e], dp[e + 1]), nd2));
+                    gk[e >> 1] = pack_bf16(f2_lo(g), f2_hi(g));
                 }
             } else {
 #pragma unroll

@@ -262,13 +262,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(scol, s);
                 tmem_ld32(scol + 32, s + 32);
                 tmem_wait_ld();
+                // 8 chains of three-input max: 28 instructions for 56 values
                 float mx8[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) mx8[e] = s[e];
 #pragma unroll
-                for (int k = 8; k < 64; ++k) mx8[k & 7] = fmaxf(mx8[k & 7], s[k]);
-                pmax = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                for (int k = 8; k < 64; k += 2) mx8[(k >> 1) & 7] = fmax3(mx8[(k >> 1) & 7], s[k], s[k + 1]);
+                pmax = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmaxf(mx8[6], mx8[7]));
             }
             // row maximum over both halves
             red[((t & 1) * 2 + g) * 128 + r] = pmax;
@@ -301,17 +302,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             uint32_t pk[32];
             if (valid) {
-                float ls8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ls8[e] = 0.f;
+                // pairs of keys: the exponent s c - m of each is one packed
+                // fused multiply-add; four packed partial sums
+                const uint64_t c2 = f2_pack(c, c), nm2 = f2_pack(-m, -m);
+                uint64_t ls2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int k = 0; k < 64; k += 2) {
-                    const float p0 = fast_exp2(fmaf(s[k], c, -m));
-                    const float p1 = fast_exp2(fmaf(s[k + 1], c, -m));
-                    ls8[(k >> 1) & 7] += p0 + p1;
+                    const uint64_t x = f2_fma(f2_pack(s[k], s[k + 1]), c2, nm2);
+                    const float p0 = fast_exp2(f2_lo(x));
+                    const float p1 = fast_exp2(f2_hi(x));
+                    ls2[(k >> 1) & 3] = f2_add(ls2[(k >> 1) & 3], f2_pack(p0, p1));
                     pk[k >> 1] = pack_bf16(p0, p1);
                 }
-                l += ((ls8[0] + ls8[1]) + (ls8[2] + ls8[3])) + ((ls8[4] + ls8[5]) + (ls8[6] + ls8[7]));
+                const uint64_t lsum = f2_add(f2_add(ls2[0], ls2[1]), f2_add(ls2[2], ls2[3]));
+                l += f2_lo(lsum) + f2_hi(lsum);
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) pk[e] = 0u;
