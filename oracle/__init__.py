@@ -55,6 +55,9 @@ def _declare(L):
                                   _P, _P, _P, _P, _P, _P, _P, _P]
     L.oracle_scores_f32.restype = None
     L.oracle_scores_f32.argtypes = [_P, _P, _I64, _I64, _I, _F, _P]
+    L.oracle_mask_from_scores.restype = None
+    L.oracle_mask_from_scores.argtypes = [_P, _I64, _I64, _I, _I, _F, _I, _I, _I, _U,
+                                          _P, _P, _P, _P, _P, _P, _P]
     L.oracle_mask.restype = None
     L.oracle_mask.argtypes = [_P, _P, _I64, _I64, _I, _I, _I, _F, _F, _I, _I, _I, _U,
                               _P, _P, _P, _P, _P, _P, _P]
@@ -178,6 +181,24 @@ def mask(qbar, kbar, grid, p, scale, window=(3, 3, 3), flags=0, cols=True):
                       np.float32(scale), *window, flags, _ptr(m["bits"]), _ptr(m["row_idx"]),
                       _ptr(m["row_cnt"]), _ptr(m.get("col_idx")), _ptr(m.get("col_cnt")),
                       _ptr(m["adapt_cnt"]), _ptr(m["margin"]))
+    return m
+
+
+def mask_from_scores(scores, grid, p, window=(3, 3, 3), flags=0, cols=True):
+    """Mask in decision precision from given float32 score rows [BH, nb, nb]
+    (for instance the scores a kernel reports): the same cut, STA and
+    diagonal as mask(), applied to those values."""
+    scores = _c(scores, np.float32)
+    BH, nb, nb2 = scores.shape
+    assert nb == nb2
+    T, Hp, Wp = grid
+    assert T * Hp * Wp == nb
+    m = _mask_buffers(BH, nb, cols)
+    m["margin"] = np.zeros((BH, nb), dtype=np.float64)
+    lib().oracle_mask_from_scores(_ptr(scores), BH, nb, Hp, Wp, np.float32(p), *window, flags,
+                                  _ptr(m["bits"]), _ptr(m["row_idx"]), _ptr(m["row_cnt"]),
+                                  _ptr(m.get("col_idx")), _ptr(m.get("col_cnt")),
+                                  _ptr(m["adapt_cnt"]), _ptr(m["margin"]))
     return m
 
 

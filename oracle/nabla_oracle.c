@@ -327,25 +327,63 @@ static int64_t cut_row_fixed(const float *score, int64_t nb, float p, uint8_t *k
     return k;
 }
 
-/* Block scores in decision precision: s = fmaf chain over d = 0..D-1 starting
- * from 0, then s * scale in float32.  qbar/kbar: [BH, nb, D] float32. */
+/* Block scores of one query block in decision precision (bullet
+ * "縮小されたアテンション": the attention map over the pooled blocks):
+ *   s_j = (fmaf chain over d = 0..D-1 of qi[d] * kbar_j[d], starting from 0)
+ *         * scale,
+ * every operation in float32.  kbar_bh: [nb, D] float32 of the same head. */
+static void scores_row_f32(const float *qi, const float *kbar_bh, int64_t nb, int D, float scale,
+                           float *score)
+{
+    for (int64_t j = 0; j < nb; ++j) {
+        const float *kj = kbar_bh + j * D;
+        float s = 0.0f;
+        for (int d = 0; d < D; ++d) s = fmaf(qi[d], kj[d], s);
+        score[j] = s * scale;
+    }
+}
+
+/* All block scores, qbar/kbar: [BH, nb, D] float32 -> scores [BH, nb, nb]. */
 void oracle_scores_f32(const float *qbar, const float *kbar, int64_t BH, int64_t nb, int D,
-                       float scale, float *scores /* [BH, nb, nb] */)
+                       float scale, float *scores)
 {
 #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t bh = 0; bh < BH; ++bh)
-        for (int64_t i = 0; i < nb; ++i) {
-            const float *qi = qbar + (bh * nb + i) * D;
-            for (int64_t j = 0; j < nb; ++j) {
-                const float *kj = kbar + (bh * nb + j) * D;
-                float s = 0.0f;
-                for (int d = 0; d < D; ++d) s = fmaf(qi[d], kj[d], s);
-                scores[(bh * nb + i) * nb + j] = s * scale;
-            }
-        }
+        for (int64_t i = 0; i < nb; ++i)
+            scores_row_f32(qbar + (bh * nb + i) * D, kbar + bh * nb * D, nb, D, scale,
+                           scores + (bh * nb + i) * nb);
 }
 
-/* Mask in decision precision from float32 pooled means (oracle_pool_f32). */
+/* Mask in decision precision from given float32 score rows [BH, nb, nb]:
+ * the cut of cut_row_fixed on each row, then OR with STA and the diagonal. */
+void oracle_mask_from_scores(const float *scores, int64_t BH, int64_t nb, int Hp, int Wp,
+                             float p, int wt, int wh, int ww, unsigned flags, uint32_t *bits,
+                             uint16_t *row_idx, int32_t *row_cnt, uint16_t *col_idx,
+                             int32_t *col_cnt, int32_t *adapt_cnt, double *margin)
+{
+    uint8_t *keep_all = (uint8_t *)malloc((size_t)(BH * nb * nb));
+#pragma omp parallel
+    {
+        uint64_t *u = (uint64_t *)malloc(sizeof(uint64_t) * (size_t)nb);
+        rank_item *scratch = (rank_item *)malloc(sizeof(rank_item) * (size_t)nb);
+#pragma omp for schedule(dynamic, 16)
+        for (int64_t r = 0; r < BH * nb; ++r) {
+            double mg;
+            int64_t k = cut_row_fixed(scores + r * nb, nb, p, keep_all + r * nb, scratch, u, &mg);
+            if (adapt_cnt) adapt_cnt[r] = (int32_t)k;
+            if (margin) margin[r] = mg;
+        }
+        free(u);
+        free(scratch);
+    }
+    emit_mask(keep_all, BH, nb, Hp, Wp, wt, wh, ww, flags, bits, row_idx, row_cnt, col_idx,
+              col_cnt);
+    free(keep_all);
+}
+
+/* Mask in decision precision from float32 pooled means (oracle_pool_f32):
+ * scores_row_f32 then cut_row_fixed on every row, then OR with STA and the
+ * diagonal. */
 void oracle_mask(const float *qbar, const float *kbar, int64_t BH, int64_t nb, int D, int Hp,
                  int Wp, float p, float scale, int wt, int wh, int ww, unsigned flags,
                  uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt, uint16_t *col_idx,
@@ -360,13 +398,8 @@ void oracle_mask(const float *qbar, const float *kbar, int64_t BH, int64_t nb, i
 #pragma omp for collapse(2) schedule(dynamic, 16)
         for (int64_t bh = 0; bh < BH; ++bh)
             for (int64_t i = 0; i < nb; ++i) {
-                const float *qi = qbar + (bh * nb + i) * D;
-                for (int64_t j = 0; j < nb; ++j) {
-                    const float *kj = kbar + (bh * nb + j) * D;
-                    float s = 0.0f;
-                    for (int d = 0; d < D; ++d) s = fmaf(qi[d], kj[d], s);
-                    score[j] = s * scale;
-                }
+                scores_row_f32(qbar + (bh * nb + i) * D, kbar + bh * nb * D, nb, D, scale,
+                               score);
                 double mg;
                 int64_t k = cut_row_fixed(score, nb, p, keep_all + (bh * nb + i) * nb, scratch,
                                           u, &mg);
