@@ -11,12 +11,12 @@
 // launchers (mask.cu, flatten.cu, attn_*.cu)
 cudaError_t nabla_launch_flatten(const void *in, void *out, int64_t outer, int T, int H, int W,
                                  int P, int64_t inner_bytes, int inverse, cudaStream_t stream);
-cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int Hp, int Wp, float p,
+cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, int Wp, float p,
                                     float scale, int wt, int wh, int ww, unsigned flags,
                                     const void *q, const void *k, float *qbar, float *kbar_t,
                                     uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
-                                    uint16_t *col_idx, int32_t *col_cnt, cudaStream_t stream,
-                                    const void *q_grid, const void *k_grid);
+                                    uint16_t *col_idx, int32_t *col_cnt, float *scores,
+                                    cudaStream_t stream, const void *q_grid, const void *k_grid);
 cudaError_t nabla_launch_attn_fwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
                                       const void *k, const void *v, const uint16_t *row_idx,
                                       const int32_t *row_cnt, void *o, float *lse,
@@ -79,7 +79,8 @@ int check_params(const nabla_params *p, bool need_window) {
     if (p == nullptr) return NABLA_ERR_NULL;
     if (!(p->p >= 0.f && p->p <= 1.f)) return NABLA_ERR_PARAM;  // also rejects NaN
     if (!(p->scale > 0.f) || !std::isfinite(p->scale)) return NABLA_ERR_PARAM;
-    if ((p->flags & ~(NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS | NABLA_DEBUG_TIMEOUT)) != 0)
+    if ((p->flags & ~(NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS | NABLA_DEBUG_SCORES |
+                      NABLA_DEBUG_TIMEOUT)) != 0)
         return NABLA_ERR_PARAM;
     if ((p->flags & NABLA_NO_STA) && (p->flags & NABLA_FULL_STA)) return NABLA_ERR_PARAM;
     if (need_window && !(p->flags & (NABLA_NO_STA | NABLA_FULL_STA))) {
@@ -124,6 +125,26 @@ int clear_status(void *ws, cudaStream_t s) {
     return cuda_status(cudaMemsetAsync(ws, 0, sizeof(int), s));
 }
 
+bool overlap(const void *a, const void *b, size_t bytes) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + bytes && y < x + bytes;
+}
+
+// Pointer checks shared by the three mask-building calls.
+int check_mask_ptrs(const nabla_params *params, const nabla_mask *mask) {
+    if (mask == nullptr || mask->bits == nullptr || mask->row_idx == nullptr ||
+        mask->row_cnt == nullptr)
+        return NABLA_ERR_NULL;
+    if ((params->flags & NABLA_EMIT_COLS) && (mask->col_idx == nullptr || mask->col_cnt == nullptr))
+        return NABLA_ERR_NULL;
+    if ((params->flags & NABLA_DEBUG_SCORES) && mask->scores == nullptr) return NABLA_ERR_NULL;
+    return NABLA_OK;
+}
+
+float *debug_scores(const nabla_params *params, const nabla_mask *mask) {
+    return (params->flags & NABLA_DEBUG_SCORES) ? mask->scores : nullptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -136,7 +157,8 @@ int nabla_flatten(const void *in, void *out, int64_t outer, int T, int H, int W,
     if (outer == 0 || T == 0 || H == 0 || W == 0 || inner_bytes == 0) return NABLA_OK;  // empty
     if (in == nullptr || out == nullptr) return NABLA_ERR_NULL;
     if (!aligned16(in) || !aligned16(out)) return NABLA_ERR_ALIGN;
-    if (in == out) return NABLA_ERR_PARAM;
+    const size_t bytes = static_cast<size_t>(outer) * T * H * W * static_cast<size_t>(inner_bytes);
+    if (overlap(in, out, bytes)) return NABLA_ERR_PARAM;
     return cuda_status(nabla_launch_flatten(in, out, outer, T, H, W, P, inner_bytes, inverse,
                                             reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -160,6 +182,8 @@ size_t nabla_mask_bytes(const nabla_shape *shape, int part) {
         case NABLA_MASK_ROW_CNT:
         case NABLA_MASK_COL_CNT:
             return rows * sizeof(int32_t);
+        case NABLA_MASK_SCORES:
+            return rows * d.nb * sizeof(float);
         default:
             return 0;
     }
@@ -172,11 +196,9 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params, const
     int st = check_shape(shape, &d);
     if (st != NABLA_OK) return st;
     if ((st = check_params(params, true)) != NABLA_OK) return st;
-    if (q == nullptr || k == nullptr || mask == nullptr || mask->bits == nullptr ||
-        mask->row_idx == nullptr || mask->row_cnt == nullptr)
-        return NABLA_ERR_NULL;
+    if (q == nullptr || k == nullptr) return NABLA_ERR_NULL;
+    if ((st = check_mask_ptrs(params, mask)) != NABLA_OK) return st;
     const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
-    if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k)) return NABLA_ERR_ALIGN;
     if ((st = check_ws(d, NABLA_OP_BUILD_MASK, workspace, workspace_bytes)) != NABLA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -185,18 +207,11 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params, const
     float *qbar = reinterpret_cast<float *>(w);
     float *kbar_t = reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
-        d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
-        params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
-        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr, s,
-        nullptr, nullptr));
+        d.BH, d.nb, d.D, shape->T, d.Hp, d.Wp, params->p, params->scale, params->sta_t,
+        params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
+        mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
+        cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, nullptr, nullptr));
 }
-
-namespace {
-bool overlap(const void *a, const void *b, size_t bytes) {
-    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
-    return x < y + bytes && y < x + bytes;
-}
-}  // namespace
 
 int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
                           const nabla_bf16 *q_grid, const nabla_bf16 *k_grid, nabla_bf16 *q,
@@ -206,12 +221,10 @@ int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
     int st = check_shape(shape, &d);
     if (st != NABLA_OK) return st;
     if ((st = check_params(params, true)) != NABLA_OK) return st;
-    if (q_grid == nullptr || k_grid == nullptr || q == nullptr || k == nullptr ||
-        mask == nullptr || mask->bits == nullptr || mask->row_idx == nullptr ||
-        mask->row_cnt == nullptr)
+    if (q_grid == nullptr || k_grid == nullptr || q == nullptr || k == nullptr)
         return NABLA_ERR_NULL;
+    if ((st = check_mask_ptrs(params, mask)) != NABLA_OK) return st;
     const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
-    if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
     if (!aligned16(q_grid) || !aligned16(k_grid) || !aligned16(q) || !aligned16(k))
         return NABLA_ERR_ALIGN;
     // the flattened outputs must not overlap each other or either input
@@ -226,10 +239,10 @@ int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
     float *qbar = reinterpret_cast<float *>(w);
     float *kbar_t = reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
-        d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
-        params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
-        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr, s, q_grid,
-        k_grid));
+        d.BH, d.nb, d.D, shape->T, d.Hp, d.Wp, params->p, params->scale, params->sta_t,
+        params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
+        mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
+        cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, q_grid, k_grid));
 }
 
 int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
@@ -361,11 +374,9 @@ extern "C" int nabla_build_mask_static(const nabla_shape *shape, const nabla_par
     int st = check_shape(shape, &d);
     if (st != NABLA_OK) return st;
     if ((st = check_params(params, true)) != NABLA_OK) return st;
-    if (q == nullptr || k == nullptr || mask == nullptr || mask->bits == nullptr ||
-        mask->row_idx == nullptr || mask->row_cnt == nullptr)
-        return NABLA_ERR_NULL;
+    if (q == nullptr || k == nullptr) return NABLA_ERR_NULL;
+    if ((st = check_mask_ptrs(params, mask)) != NABLA_OK) return st;
     const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
-    if (cols && (mask->col_idx == nullptr || mask->col_cnt == nullptr)) return NABLA_ERR_NULL;
     if (!aligned16(q) || !aligned16(k)) return NABLA_ERR_ALIGN;
     const MaskScratch ms = mask_scratch(d);
     if (ms.qbar_bytes + ms.kbar_bytes > kStaticScratchBytes) return NABLA_ERR_WORKSPACE;
@@ -376,8 +387,9 @@ extern "C" int nabla_build_mask_static(const nabla_shape *shape, const nabla_par
     float *qbar = static_cast<float *>(base);
     float *kbar_t = reinterpret_cast<float *>(static_cast<unsigned char *>(base) + ms.qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
-        d.BH, d.nb, d.D, d.Hp, d.Wp, params->p, params->scale, params->sta_t, params->sta_h,
-        params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits, mask->row_idx,
-        mask->row_cnt, cols ? mask->col_idx : nullptr, cols ? mask->col_cnt : nullptr,
+        d.BH, d.nb, d.D, shape->T, d.Hp, d.Wp, params->p, params->scale, params->sta_t,
+        params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
+        mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
+        cols ? mask->col_cnt : nullptr, debug_scores(params, mask),
         reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr));
 }

@@ -15,9 +15,9 @@ LIB_PATH = os.path.join(HERE, "libnabla.so")
 OK = 0
 ERR_SHAPE, ERR_ALIGN, ERR_PARAM, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_NULL = (
     -1, -2, -3, -4, -5, -6, -7)
-NO_STA, FULL_STA, EMIT_COLS, DEBUG_TIMEOUT = 1, 2, 4, 0x100
+NO_STA, FULL_STA, EMIT_COLS, DEBUG_SCORES, DEBUG_TIMEOUT = 1, 2, 4, 8, 0x100
 OP_BUILD_MASK, OP_ATTN_FWD, OP_ATTN_BWD = 0, 1, 2
-MASK_BITS, MASK_ROW_IDX, MASK_ROW_CNT, MASK_COL_IDX, MASK_COL_CNT = 0, 1, 2, 3, 4
+MASK_BITS, MASK_ROW_IDX, MASK_ROW_CNT, MASK_COL_IDX, MASK_COL_CNT, MASK_SCORES = 0, 1, 2, 3, 4, 5
 
 # every symbol include/nabla.h declares
 SYMBOLS = ("nabla_flatten", "nabla_workspace_size", "nabla_mask_bytes", "nabla_build_mask",
@@ -41,7 +41,8 @@ class Params(ctypes.Structure):
 
 
 class MaskStruct(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("bits", "row_idx", "row_cnt", "col_idx", "col_cnt")]
+    _fields_ = [(n, ctypes.c_void_p)
+                for n in ("bits", "row_idx", "row_cnt", "col_idx", "col_cnt", "scores")]
 
 
 _lib = None
@@ -128,7 +129,7 @@ def workspace(shape, op, device):
     return torch.empty(n, dtype=torch.uint8, device=device)
 
 
-def alloc_mask(shape, device, cols=True):
+def alloc_mask(shape, device, cols=True, scores=False):
     BH, nb = shape.B * shape.heads, shape.T * (shape.H // shape.P) * (shape.W // shape.P)
     words = (nb + 31) // 32
     m = {"bits": torch.empty((BH, nb, words), dtype=torch.int32, device=device),
@@ -137,8 +138,11 @@ def alloc_mask(shape, device, cols=True):
     if cols:
         m["col_idx"] = torch.empty((BH, nb, nb), dtype=torch.int16, device=device)
         m["col_cnt"] = torch.empty((BH, nb), dtype=torch.int32, device=device)
+    if scores:
+        m["scores"] = torch.empty((BH, nb, nb), dtype=torch.float32, device=device)
     for part, key in ((MASK_BITS, "bits"), (MASK_ROW_IDX, "row_idx"), (MASK_ROW_CNT, "row_cnt"),
-                      (MASK_COL_IDX, "col_idx"), (MASK_COL_CNT, "col_cnt")):
+                      (MASK_COL_IDX, "col_idx"), (MASK_COL_CNT, "col_cnt"),
+                      (MASK_SCORES, "scores")):
         if key in m:
             assert m[key].numel() * m[key].element_size() == mask_bytes(shape, part)
     return m
@@ -146,7 +150,7 @@ def alloc_mask(shape, device, cols=True):
 
 def _mask_struct(m):
     return MaskStruct(*(_ptr(m.get(k)) for k in ("bits", "row_idx", "row_cnt", "col_idx",
-                                                  "col_cnt")))
+                                                  "col_cnt", "scores")))
 
 
 def flatten(x, T, H, W, P=8, inverse=False, out=None):
@@ -167,7 +171,8 @@ def build_mask(shape, params, q, k, mask=None, ws=None):
     _need(q, torch.bfloat16, "q")
     _need(k, torch.bfloat16, "k")
     cols = bool(params.flags & EMIT_COLS)
-    mask = alloc_mask(shape, q.device, cols) if mask is None else mask
+    dbg = bool(params.flags & DEBUG_SCORES)
+    mask = alloc_mask(shape, q.device, cols, dbg) if mask is None else mask
     ws = workspace(shape, OP_BUILD_MASK, q.device) if ws is None else ws
     ms = _mask_struct(mask)
     _check(lib().nabla_build_mask(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k),
@@ -184,7 +189,8 @@ def build_mask_grid(shape, params, q_grid, k_grid, q=None, k=None, mask=None, ws
     q = torch.empty_like(q_grid) if q is None else q
     k = torch.empty_like(k_grid) if k is None else k
     cols = bool(params.flags & EMIT_COLS)
-    mask = alloc_mask(shape, q_grid.device, cols) if mask is None else mask
+    dbg = bool(params.flags & DEBUG_SCORES)
+    mask = alloc_mask(shape, q_grid.device, cols, dbg) if mask is None else mask
     ws = workspace(shape, OP_BUILD_MASK, q_grid.device) if ws is None else ws
     ms = _mask_struct(mask)
     _check(lib().nabla_build_mask_grid(ctypes.byref(shape), ctypes.byref(params), _ptr(q_grid),

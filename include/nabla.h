@@ -15,7 +15,10 @@
  * Conventions shared by every call
  *   - All tensors live in device memory that the CALLER allocated; the library
  *     allocates nothing and keeps no state between calls.  Scratch memory is
- *     the caller's workspace, sized by nabla_workspace_size().
+ *     the caller's workspace, sized by nabla_workspace_size().  The one
+ *     exception is nabla_build_mask_static, whose scratch is an array compiled
+ *     into the library (held per GPU until exit) and which caches that array's
+ *     device address per device.
  *   - Every call only enqueues work on `stream` (a cudaStream_t; NULL is the
  *     legacy default stream) and returns without synchronising the host.
  *     Errors found on the host (shape, alignment, parameters, workspace size,
@@ -56,6 +59,11 @@ typedef struct CUstream_st *nabla_stream_t; /* == cudaStream_t */
 #define NABLA_NO_STA 1u    /* no STA term: M = adaptive OR diagonal            */
 #define NABLA_FULL_STA 2u  /* STA window covers every block: dense attention   */
 #define NABLA_EMIT_COLS 4u /* also write the column lists needed by the backward */
+/* Also write the pooled block scores s_ij (float32, [B*heads, nb, nb]) into
+ * mask->scores, exactly as the cut used them, so that a caller can re-run the
+ * cut on them (a check of the score phase).  Written only when the mask
+ * depends on the scores (0 < p < 1 and not NABLA_FULL_STA). */
+#define NABLA_DEBUG_SCORES 8u
 /* Test aid, not for production: makes the tensor-core attention forward and
  * backward (D = 128) give up a device-side wait at once, so that the timeout
  * path (status word = NABLA_ERR_TIMEOUT, clean unwind, context still usable)
@@ -77,7 +85,8 @@ typedef struct {
  *          patch columns), centred, truncated at the grid border.
  *   scale  softmax scale of both the pooled map and the attention
  *          (usually 1/sqrt(D)).
- *   flags  NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS. */
+ *   flags  NABLA_NO_STA | NABLA_FULL_STA | NABLA_EMIT_COLS |
+ *          NABLA_DEBUG_SCORES (and the test aid NABLA_DEBUG_TIMEOUT). */
 typedef struct {
     float p;
     int sta_t, sta_h, sta_w;
@@ -93,13 +102,16 @@ typedef struct {
  *   row_cnt [B*heads, nb] int32.
  *   col_idx, col_cnt: the transpose (query blocks i keeping key block j,
  *           ascending i); written only with NABLA_EMIT_COLS, required by
- *           nabla_attn_bwd.  May be NULL otherwise. */
+ *           nabla_attn_bwd.  May be NULL otherwise.
+ *   scores  [B*heads, nb, nb] float32 pooled scores; written only with
+ *           NABLA_DEBUG_SCORES (then required), may be NULL otherwise. */
 typedef struct {
     uint32_t *bits;
     uint16_t *row_idx;
     int32_t *row_cnt;
     uint16_t *col_idx;
     int32_t *col_cnt;
+    float *scores;
 } nabla_mask;
 
 /* Which part of the mask nabla_mask_bytes() sizes. */
@@ -108,6 +120,7 @@ typedef struct {
 #define NABLA_MASK_ROW_CNT 2
 #define NABLA_MASK_COL_IDX 3
 #define NABLA_MASK_COL_CNT 4
+#define NABLA_MASK_SCORES 5
 
 /* Which call nabla_workspace_size() sizes. */
 #define NABLA_OP_BUILD_MASK 0
@@ -121,9 +134,9 @@ typedef struct {
  *   n = ((t*(H/P) + y/P)*(W/P) + x/P)*P*P + (y%P)*P + x%P
  * (one level of P x P patches, patch grid and patch interior row-major).
  * inverse = 0 maps grid -> flattened, inverse = 1 flattened -> grid.
- * Any P >= 1 dividing H and W; inner_bytes % 16 == 0; in != out (no
- * in-place).  Works for [B, T, H, W, C] activations and [B*h, T, H, W, D]
- * heads alike. */
+ * Any P >= 1 dividing H and W; inner_bytes % 16 == 0; in and out must not
+ * overlap (NABLA_ERR_PARAM; no in-place).  Works for [B, T, H, W, C]
+ * activations and [B*h, T, H, W, D] heads alike. */
 int nabla_flatten(const void *in, void *out, int64_t outer, int T, int H, int W, int P,
                   int64_t inner_bytes, int inverse, nabla_stream_t stream);
 
@@ -145,7 +158,8 @@ size_t nabla_mask_bytes(const nabla_shape *shape, int part);
  *   adaptive set   = shortest prefix of j ordered by (s_ij desc, j asc) whose
  *                    summed u reaches p * sum_j u_ij (float64 product);
  *   M_ij           = adaptive OR STA window OR (i == j).
- * Writes bits, row lists, and (with NABLA_EMIT_COLS) column lists.
+ * Writes bits, row lists, (with NABLA_EMIT_COLS) column lists and (with
+ * NABLA_DEBUG_SCORES) the scores s_ij.
  * When M does not depend on the scores -- p >= 1 or NABLA_FULL_STA (every
  * block), p <= 0 (STA window and diagonal; the diagonal alone with
  * NABLA_NO_STA) -- q and k are not read and no pooling or scores are computed
@@ -194,6 +208,8 @@ int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
  *     contents.  Calls whose GPU work overlaps (other streams, other host
  *     threads) race on it; serialise them.  Nothing in the array needs to
  *     start at zero: each call writes every scratch byte it reads.
+ *   - cudaDeviceReset invalidates the cached address: after resetting a
+ *     device, do not call this entry point on it again in the same process.
  * Other arguments, checks and outputs: as nabla_build_mask. */
 int nabla_build_mask_static(const nabla_shape *shape, const nabla_params *params,
                             const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,

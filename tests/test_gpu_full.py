@@ -64,10 +64,50 @@ def test_720p_mask_every_row(train720):
     assert check_mask(gm, om) == 0
 
 
+def test_720p_debug_scores_cut_only(train720):
+    """The kernel's own float32 scores (NABLA_DEBUG_SCORES) equal the oracle's
+    score routine bit for bit, and the oracle's cut applied to them gives the
+    kernel's mask on every row of all 40 heads."""
+    c = train720
+    prm = c.params(c.p, nabla.DEBUG_SCORES)
+    gm = to_np(nabla.build_mask(c.shape, prm, c.gpu["q"], c.gpu["k"]))
+    qb, kb = oracle.pool_f32(c.cpu["q"]), oracle.pool_f32(c.cpu["k"])
+    assert np.array_equal(gm["scores"], oracle.scores_f32(qb, kb, c.w.scale))
+    om = oracle.mask_from_scores(gm["scores"], c.w.grid_blocks, c.p, c.w.window)
+    assert check_mask(gm, om) == 0
+
+
 def test_720p_forward_sampled(train720):
     om = train720.oracle_mask()
     gm = train720.gpu_mask()
     _sampled_forward(train720, om, gm, heads=(0, 17, 39), blocks_per_head=32, seed=1)
+
+
+def _key_pairs(w, col_idx, col_cnt, rng, pairs=4):
+    """Key blocks for the sampled dK/dV check of one head: `pairs` temporal
+    pairs (the same patch in frames 2u and 2u + 1, the unit the dK/dV kernel
+    walks together), spatial neighbours of each other so that their column
+    lists overlap, plus the pair among a seeded candidate set whose two column
+    lists differ the most (the union the kernel walks is then not one list)."""
+    T, Hp, Wp = w.grid_blocks
+    hw = Hp * Wp
+
+    def pair(u, ph, pw):
+        j = (2 * u * Hp + ph) * Wp + pw
+        return j, j + hw
+
+    def diff(j0, j1):
+        a = set(col_idx[j0, :col_cnt[j0]].tolist())
+        b = set(col_idx[j1, :col_cnt[j1]].tolist())
+        return len(a ^ b)
+
+    u, ph, pw = int(rng.integers(T // 2)), int(rng.integers(Hp - 1)), int(rng.integers(Wp - 1))
+    out = list(pair(u, ph, pw)) + list(pair(u, ph, pw + 1)) + list(pair(u, ph + 1, pw))
+    cands = [pair(int(rng.integers(T // 2)), int(rng.integers(Hp)), int(rng.integers(Wp)))
+             for _ in range(24)]
+    out += list(max(cands, key=lambda jj: diff(*jj)))
+    assert diff(out[-2], out[-1]) > 0
+    return out[:2 * pairs]
 
 
 def test_720p_backward_sampled(train720):
@@ -82,9 +122,10 @@ def test_720p_backward_sampled(train720):
     x = _heads_f64(c, ("q", "k", "v", "dout"), heads)
     sm = _slice_mask(om, heads)
     rng = np.random.default_rng(2)
-    dq_sel = [(hh, int(i)) for hh in range(2) for i in rng.choice(w.nb, 8, replace=False)]
-    j0 = int(rng.integers(w.nb - 1))
-    kv_sel = [(0, j0), (0, j0 + 1)]  # neighbours: their column lists overlap
+    dq_sel = [(hh, int(i)) for hh in range(2) for i in rng.choice(w.nb, 6, replace=False)]
+    kv_sel = [(hh, j) for hh in range(2) for j in _key_pairs(w, sm["col_idx"][hh],
+                                                             sm["col_cnt"][hh], rng)]
+    assert len(kv_sel) == 16
     oq, ok_, ov = oracle.attn_bwd(x["q"], x["k"], x["v"], x["dout"], sm["row_idx"],
                                   sm["row_cnt"], sm["col_idx"], sm["col_cnt"], w.scale,
                                   dq_sel=dq_sel, kv_sel=kv_sel)

@@ -135,3 +135,66 @@ def test_build_mask_from_grid_matches_flatten_then_build(w, p, flags):
         raw = ws.cpu().numpy()
         qbar = raw[256:256 + 4 * n].view(np.float32).reshape(w.BH, w.nb, w.D)
         assert np.array_equal(qbar, oracle.pool_f32(c.cpu["q"]))
+
+
+# --------------------------------------------------------------------------
+# NABLA_DEBUG_SCORES: the score phase checked on its own.  The kernel's float32
+# scores must equal the oracle's score routine bit for bit, and the oracle's
+# cut (and STA, diagonal) applied to the kernel's own scores must give the
+# kernel's mask on every row.
+# --------------------------------------------------------------------------
+def _check_debug_scores(c, p, flags=0):
+    prm = c.params(p, flags | nabla.DEBUG_SCORES)
+    gm = to_np(nabla.build_mask(c.shape, prm, c.gpu["q"], c.gpu["k"]))
+    qb, kb = oracle.pool_f32(c.cpu["q"]), oracle.pool_f32(c.cpu["k"])
+    assert np.array_equal(gm["scores"], oracle.scores_f32(qb, kb, c.w.scale)), "scores differ"
+    om = oracle.mask_from_scores(gm["scores"], c.w.grid_blocks, p, c.w.window, flags)
+    assert check_mask(gm, om) == 0
+
+
+@pytest.mark.parametrize("p", [0.5, 0.8, 0.95])
+def test_debug_scores_small(small, p):
+    _check_debug_scores(small, p)
+
+
+@pytest.mark.parametrize("w", ODD, ids=lambda w: w.name)
+def test_debug_scores_ragged(w):
+    _check_debug_scores(Case(w), 0.6, nabla.NO_STA)
+
+
+# --------------------------------------------------------------------------
+# Tied scores.  The kernel ranks exactly only the histogram bucket that holds
+# the last kept block; its blocks are held in shared memory when there are at
+# most 256 of them and re-derived from the scores otherwise.  Key blocks built
+# from a few repeated patterns make whole groups of blocks tie, so both forms
+# run, and the ties are broken by block index as the definition says.
+# --------------------------------------------------------------------------
+def _repeat_k_blocks(w, patterns):
+    def mutate(inp):
+        B, h, T, H, W, D = inp["k"].shape
+        g = torch.Generator().manual_seed(11)
+        V = torch.randn(B, h, patterns, D, generator=g).to(torch.bfloat16)
+        t = torch.arange(T)[:, None, None]
+        y = torch.arange(H)[None, :, None]
+        x = torch.arange(W)[None, None, :]
+        blk = (t * (H // 8) + y // 8) * (W // 8) + x // 8           # [T, H, W]
+        inp["k"] = V[:, :, blk % patterns].contiguous()              # [B, h, T, H, W, D]
+    return mutate
+
+
+TIES = [
+    (synth.Workload("ties1_nb128", 1, 2, 8, 32, 32, 128, (2, 4, 4), 0.7), 1),     # every score equal
+    (synth.Workload("ties5_nb1200", 1, 2, 20, 48, 80, 128, (2, 8, 8), 0.7), 5),   # 240 per group
+    (synth.Workload("ties3_nb2048", 1, 1, 32, 64, 64, 128, (2, 8, 8), 0.6), 3),   # > 256 per group
+    (synth.Workload("ties1_nb600", 1, 1, 10, 48, 80, 64, (2, 8, 8), 0.45), 1),    # D = 64
+]
+
+
+@pytest.mark.parametrize("w,patterns", TIES, ids=lambda x: getattr(x, "name", str(x)))
+def test_tied_scores(w, patterns):
+    c = Case(w, mutate=_repeat_k_blocks(w, patterns))
+    for p in (0.2, w.p, 0.97):
+        gm = to_np(c.gpu_mask(p))
+        om = c.oracle_mask(p)
+        assert check_mask(gm, om) == 0
+        _check_debug_scores(c, p)

@@ -23,13 +23,13 @@ from adaptive_block_sparse_fractal_b200 import nabla, synth
 pytestmark = pytest.mark.gpu
 
 
-def _problem(w, seed):
+def _problem(w, seed, flags=nabla.EMIT_COLS):
     dev = torch.device("cuda")
     g = synth.make_inputs_device(w, seed, dev, with_dout=False)
     q = nabla.flatten(g["q"], w.T, w.H, w.W, w.P)
     k = nabla.flatten(g["k"], w.T, w.H, w.W, w.P)
     shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
-    prm = nabla.params_of(w.p, w.window, D=w.D, flags=nabla.EMIT_COLS)
+    prm = nabla.params_of(w.p, w.window, D=w.D, flags=flags)
     return shape, prm, q, k
 
 
@@ -44,9 +44,11 @@ def _static_call(shape, prm, q, k, mask):
 
 def _same(a, b):
     nb = a["row_cnt"].shape[-1]
-    for key in ("bits", "row_cnt", "col_cnt"):
+    cols = "col_cnt" in b
+    assert cols == ("col_cnt" in a)
+    for key in ("bits", "row_cnt") + (("col_cnt",) if cols else ()):
         assert torch.equal(a[key], b[key]), key
-    for idx, cnt in (("row_idx", "row_cnt"), ("col_idx", "col_cnt")):
+    for idx, cnt in (("row_idx", "row_cnt"),) + ((("col_idx", "col_cnt"),) if cols else ()):
         valid = torch.arange(nb, device=a[idx].device)[None, None, :] < a[cnt][..., None]
         assert torch.equal(torch.where(valid, a[idx], 0), torch.where(valid, b[idx], 0)), idx
 
@@ -54,10 +56,12 @@ def _same(a, b):
 def test_static_scratch_matches_workspace_entry_point_twice():
     small = synth.WORKLOADS["small"]
     odd = synth.Workload("odd130", 2, 2, 5, 16, 104, 128, (2, 4, 4), 0.7)
-    for w, seed in ((small, 0), (odd, 5)):  # two calls in a row, different shapes
-        shape, prm, q, k = _problem(w, seed)
+    tiny = synth.WORKLOADS["tiny"]  # D = 64, no column lists
+    # calls in a row, different shapes
+    for w, seed, flags in ((small, 0, nabla.EMIT_COLS), (odd, 5, nabla.EMIT_COLS), (tiny, 2, 0)):
+        shape, prm, q, k = _problem(w, seed, flags)
         want = nabla.build_mask(shape, prm, q, k)
-        got = nabla.alloc_mask(shape, q.device, cols=True)
+        got = nabla.alloc_mask(shape, q.device, cols=bool(flags & nabla.EMIT_COLS))
         for key in got:
             got[key].fill_(-1)  # stale contents must not leak into the result
         assert _static_call(shape, prm, q, k, got) == nabla.OK
