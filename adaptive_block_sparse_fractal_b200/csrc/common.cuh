@@ -59,6 +59,40 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// ---- packed two-wide float32 arithmetic (sm_100) ----------------------------
+// Each lane of the pair is rounded exactly like the scalar operation, so a
+// value computed packed equals the one computed with fmaf / + / *.  Packing
+// halves the issue slots these take, which the single-thread MMA and copy
+// issuers sharing a sub-partition with the softmax warps need.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    return (static_cast<uint64_t>(__float_as_uint(hi)) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+    return __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// max of three in one instruction (sm_100); exact, like two fmaxf
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // Byte offset of 16-byte chunk `c` of row `r` in a [rows x (chunks*16 B)]
 // shared tile whose chunks are XOR-swizzled by the row (conflict-free
 // ldmatrix over 8 consecutive rows).

@@ -191,17 +191,12 @@ __global__ void __launch_bounds__(256) flatten_pool_kernel(
 // scores + CDF cut + STA + lists
 // ---------------------------------------------------------------------------
 constexpr int kRows = 16;       // query blocks per CTA
-constexpr int kCols = 256;      // key blocks per score tile
-constexpr int kDc = 8;          // features per staged K-bar slice
-constexpr int kStages = 3;      // cp.async ring depth of the K-bar slices
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kBuckets = 256;   // mass histogram buckets of one row
-constexpr float kBucketScale = 9.0f;  // buckets per unit of (s_max - s): 256 cover 28.4
-constexpr int kWarpScratch = 2048;    // bytes per warp: histogram, then the bucket's entries
-constexpr int kListCap = kWarpScratch / 8;
-constexpr int kMaxWords = 64;   // bit-row words of the largest row (2048 blocks)
-static_assert(kStages * kDc * kCols * 4 >= kWarps * kWarpScratch, "scratch fits the ring");
+constexpr int kHistWords = 512;     // per warp: 256 bins x (hi, lo) u32
+constexpr int kMaxWords = 64;       // bit-row words of the largest row (2048 blocks)
+constexpr int kCand = 64;           // candidates ranked exactly by one warp at once
+constexpr int kPre = 16;            // features of K-bar prefetched ahead in registers
 
 struct CutParams {
     int nb, T, Hp, Wp, wt, wh, ww;
@@ -223,18 +218,21 @@ __device__ __forceinline__ uint64_t rank_key(float s, int j) {
 
 // Integer mass floor(exp(s - smax) * 2^40), held in a double (exact: an
 // integer <= 2^40; sums of up to 2^12 of them stay below 2^53, so every sum
-// below is exact whatever the order of the additions).
+// below is exact whatever the order of the additions).  s = -inf gives 0.
 __device__ __forceinline__ double mass_of(float s, float smax) {
     const double w = exp(static_cast<double>(s) - static_cast<double>(smax));
     return trunc(w * 1099511627776.0);  // * 2^40 is an exact scaling
 }
 
-// Histogram bucket of a score: non-decreasing as the score decreases (float
-// subtraction, multiplication and truncation are all monotone), equal for
-// equal scores, so the buckets cut the rank order into consecutive runs.
-__device__ __forceinline__ int bucket_of(float s, float smax) {
-    const float x = __fmul_rn(__fsub_rn(smax, s), kBucketScale);
-    return x < static_cast<float>(kBuckets) ? __float2int_rz(x) : kBuckets - 1;
+// 24-bit bucket key of a score: floor(y * 2^16) with y = (s_max - s) * g in
+// float32 (g > 0 fixed for the row), saturated at 2^24 - 1.  Float
+// subtraction and multiplication by a positive constant are monotone and
+// scaling by 2^16 is exact, so the key never decreases as the score decreases
+// and equal scores share it: its bytes, most significant first, cut the rank
+// order into consecutive runs at three levels of refinement.
+__device__ __forceinline__ uint32_t ykey(float s, float smax, float g) {
+    const float y = __fmul_rn(__fsub_rn(smax, s), g);
+    return y < 256.0f ? __float2uint_rz(__fmul_rn(y, 65536.0f)) : 0xFFFFFFu;
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -243,17 +241,35 @@ __device__ __forceinline__ double warp_sum(double v) {
     return v;
 }
 
+__device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
+    const uint32_t hi = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(v >> 32));
+    const uint32_t lo = __reduce_max_sync(
+        0xffffffffu, static_cast<uint32_t>(v >> 32) == hi ? static_cast<uint32_t>(v) : 0u);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t b, double u) {
+    const unsigned long long ui = static_cast<unsigned long long>(u);
+    atomicAdd(hist + b, static_cast<uint32_t>(ui >> 20));
+    atomicAdd(hist + 256 + b, static_cast<uint32_t>(ui & 0xFFFFFull));
+}
+
 // One CTA per (bh, 16 query blocks).
-//   Phase 1: the 16 x nb pooled scores into shared memory (register-tiled
-//            FFMA, 4 x 4 outputs per thread; K-bar^T slices of 8 features x
-//            256 blocks stream through a 3-deep cp.async ring; every output
-//            is the plain fma chain over d = 0 .. D-1).
-//   Phase 2: one warp per row.  The exact integer masses are summed into a
-//            256-bucket histogram over (s_max - s); a scan of it finds the
-//            bucket that holds the last kept block and the mass before it.
-//            Only that bucket's blocks are ranked exactly (bisection over the
-//            48-bit rank key, with the bucket's masses kept in shared memory),
-//            so no per-block state has to live in registers.
+//   Phase 1: the 16 x nb pooled scores into shared memory.  Thread t owns
+//            columns t, t + 256, ...; for each it runs the 16 rows' fma chains
+//            over d = 0 .. D-1 as packed fma.rn.f32x2 on row pairs (each lane
+//            rounds like fmaf), the query means broadcast from shared memory
+//            and the K-bar^T column read from L2 with 16 features prefetched
+//            in registers; then times scale.
+//   Phase 2: one warp per row.  Exact integer masses are summed into a
+//            256-bin histogram over the top byte of the bucket key (bins
+//            spread over the row's own score range); its scan gives the bin
+//            holding the last kept block and the mass before it.  Blocks in
+//            lower bins are kept, in higher bins dropped; the bin's own blocks
+//            are refined by the key's next byte (at most three levels) until
+//            at most 64 remain, which are ranked exactly by their 48-bit rank
+//            keys against each other.  (Runs of equal scores that no byte can
+//            split are resolved by score group, lowest index first.)
 //   Then the bit row (adaptive set OR STA window OR diagonal) and its
 //   ascending list are written.
 template <int D>
@@ -264,11 +280,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     extern __shared__ __align__(16) unsigned char smem[];
     const int nb = prm.nb;
     const int nbp = (nb + 3) & ~3;
-    float *sS = reinterpret_cast<float *>(smem);                       // [kRows][nbp]
-    float *sQt = sS + kRows * nbp;                                     // [D][kRows]
-    float *sKt = sQt + D * kRows;                                      // [kStages][kDc][kCols]
-    unsigned char *scratch = reinterpret_cast<unsigned char *>(sKt);   // phase 2, per warp
-    uint32_t *sW = reinterpret_cast<uint32_t *>(sKt + kStages * kDc * kCols);  // [kWarps][64]
+    float *sS = reinterpret_cast<float *>(smem);                  // [kRows][nbp]
+    float *sQt = sS + kRows * nbp;                                // [D][kRows]
+    uint32_t *sH = reinterpret_cast<uint32_t *>(sQt + D * kRows);  // [kWarps][kHistWords]
+    uint32_t *sW = sH + kWarps * kHistWords;                      // [kWarps][kMaxWords]
+    int *sE = reinterpret_cast<int *>(sW + kWarps * kMaxWords);   // [kWarps][kCand]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tiles = (nb + kRows - 1) / kRows;
@@ -281,65 +297,47 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int r = idx / D, d = idx % D;
         sQt[d * kRows + r] = (r < rows_here) ? qbar[(bh * nb + i0 + r) * D + d] : 0.f;
     }
-    const int cg = tid % 64;  // 4 consecutive columns
-    const int rg = tid / 64;  // 4 consecutive rows
+    __syncthreads();
     const float *kt = kbar_t + bh * static_cast<int64_t>(D) * nbp;
-    constexpr int DCH = D / kDc;  // feature slices per column tile
-    const int nstage = ((nb + kCols - 1) / kCols) * DCH;
-    auto issue = [&](int st) {
-        if (st < nstage) {
-            const int j0 = (st / DCH) * kCols, d0 = (st % DCH) * kDc;
-            float *dst = sKt + (st % kStages) * (kDc * kCols);
-            for (int c = tid; c < kDc * kCols / 4; c += kThreads) {
-                const int d = c / (kCols / 4), j = (c % (kCols / 4)) * 4;
-                float *sd = dst + d * kCols + j;
-                if (j0 + j < nbp) {
-                    cp_async16(smem_addr(sd), kt + static_cast<int64_t>(d0 + d) * nbp + j0 + j);
-                } else {
-                    *reinterpret_cast<float4 *>(sd) = make_float4(0.f, 0.f, 0.f, 0.f);
+    const uint64_t sc2 = f2_pack(prm.scale, prm.scale);
+    for (int j = tid; j < nb; j += kThreads) {
+        uint64_t acc[kRows / 2];
+#pragma unroll
+        for (int q = 0; q < kRows / 2; ++q) acc[q] = 0ull;
+        float kc[kPre], kn[kPre];
+#pragma unroll
+        for (int q = 0; q < kPre; ++q) kc[q] = __ldg(kt + static_cast<int64_t>(q) * nbp + j);
+#pragma unroll
+        for (int d0 = 0; d0 < D; d0 += kPre) {
+            if (d0 + kPre < D) {
+#pragma unroll
+                for (int q = 0; q < kPre; ++q)
+                    kn[q] = __ldg(kt + static_cast<int64_t>(d0 + kPre + q) * nbp + j);
+            }
+#pragma unroll
+            for (int q = 0; q < kPre; ++q) {
+                const float4 *qv = reinterpret_cast<const float4 *>(sQt + (d0 + q) * kRows);
+                const uint64_t kk = f2_pack(kc[q], kc[q]);
+#pragma unroll
+                for (int v = 0; v < kRows / 4; ++v) {
+                    const float4 qq = qv[v];
+                    acc[2 * v] = f2_fma(f2_pack(qq.x, qq.y), kk, acc[2 * v]);
+                    acc[2 * v + 1] = f2_fma(f2_pack(qq.z, qq.w), kk, acc[2 * v + 1]);
                 }
             }
+            if (d0 + kPre < D) {
+#pragma unroll
+                for (int q = 0; q < kPre; ++q) kc[q] = kn[q];
+            }
         }
-        cp_async_commit();  // an empty group past the end keeps the counting uniform
-    };
-    float acc[4][4];
-    issue(0);
-    issue(1);
-    for (int st = 0; st < nstage; ++st) {
-        cp_async_wait<1>();  // slice st has landed (only st + 1 may be in flight)
-        __syncthreads();     // ... for every thread; slot (st + 2) % 3 is free again
-        issue(st + 2);
-        const int j0 = (st / DCH) * kCols, d0 = (st % DCH) * kDc;
-        if (d0 == 0) {
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-        }
-        const float *sk = sKt + (st % kStages) * (kDc * kCols);
-#pragma unroll
-        for (int d = 0; d < kDc; ++d) {
-            const float4 qv = *reinterpret_cast<const float4 *>(sQt + (d0 + d) * kRows + rg * 4);
-            const float4 kv = *reinterpret_cast<const float4 *>(sk + d * kCols + cg * 4);
-            const float qa[4] = {qv.x, qv.y, qv.z, qv.w};
-            const float ka[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) acc[a][b] = __fmaf_rn(qa[a], ka[b], acc[a][b]);
-        }
-        if (d0 + kDc == D) {
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    const int j = j0 + cg * 4 + b;
-                    if (j < nb) sS[(rg * 4 + a) * nbp + j] = __fmul_rn(acc[a][b], prm.scale);
-                }
+        for (int q = 0; q < kRows / 2; ++q) {
+            const uint64_t a = f2_mul(acc[q], sc2);
+            sS[(2 * q) * nbp + j] = f2_lo(a);
+            sS[(2 * q + 1) * nbp + j] = f2_hi(a);
         }
     }
-    cp_async_wait<0>();
-    __syncthreads();  // scores complete; the ring becomes the warps' scratch
+    __syncthreads();  // scores complete
 
     if (scores_out != nullptr) {  // NABLA_DEBUG_SCORES: the rows as computed
         for (int idx = tid; idx < rows_here * nb; idx += kThreads) {
@@ -351,152 +349,230 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- phase 2: one warp per row
     const int words = (nb + 31) >> 5;
     const unsigned lt = (1u << lane) - 1u;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(scratch + warp * kWarpScratch);  // hi | lo
-    unsigned long long *ent = reinterpret_cast<unsigned long long *>(scratch + warp * kWarpScratch);
+    uint32_t *hist = sH + warp * kHistWords;  // hi[256] | lo[256]
     uint32_t *sw = sW + warp * kMaxWords;
+    int *ent = sE + warp * kCand;
     const int HWp = prm.Hp * prm.Wp;
     for (int r = warp; r < rows_here; r += kWarps) {
         const int i = i0 + r;
         const float *srow = sS + r * nbp;
+        auto score = [&](int j) { return j < nb ? srow[j] : -INFINITY; };
+        auto clear_hist = [&]() {
+            uint4 *h4 = reinterpret_cast<uint4 *>(hist);
+            for (int k = lane; k < kHistWords / 4; k += 32) h4[k] = make_uint4(0u, 0u, 0u, 0u);
+        };
 
-        // row maximum
-        float smax = -INFINITY;
-        for (int j = lane; j < nb; j += 32) smax = fmaxf(smax, srow[j]);
+        // row maximum and minimum
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float mn[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+        for (int e0 = 0; e0 < words; e0 += 4) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+            for (int u = 0; u < 4; ++u) {
+                const int j = (e0 + u) * 32 + lane;
+                if (j < nb) {
+                    const float s = srow[j];
+                    mx[u] = fmaxf(mx[u], s);
+                    mn[u] = fminf(mn[u], s);
+                }
+            }
+        }
+        float smax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        float smin = fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3]));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+            smin = fminf(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+        }
+        // bins over [0, span) of s_max - s; beyond 28 the masses are 0
+        // (e^-28 * 2^40 < 1), so those blocks may share the last bin
+        const float span = fminf(fmaxf(__fsub_rn(smax, smin), 0.0009765625f), 28.0f);
+        const float g = __fdiv_rn(256.0f, span);
 
-        // mass histogram: bucket b gets hi = sum (u >> 20) and lo = sum (u & (2^20 - 1));
-        // each sum stays below 2^31 for up to 2048 blocks, so the u32 adds are exact
-        for (int k = lane; k < 2 * kBuckets; k += 32) hist[k] = 0u;
+        // level 0: every block's mass into the bin of its key's top byte, and
+        // the row total.  The bins hold hi = sum (u >> 20) and lo = sum (u &
+        // (2^20 - 1)); each stays below 2^31 for up to 2048 blocks (exact).
+        clear_hist();
         __syncwarp();
         double U = 0.0;
-        for (int j = lane; j < nb; j += 32) {
-            const float s = srow[j];
-            const double u = mass_of(s, smax);
-            if (u > 0.0) {
-                const unsigned long long ui = static_cast<unsigned long long>(u);
-                const int b = bucket_of(s, smax);
-                atomicAdd(hist + b, static_cast<uint32_t>(ui >> 20));
-                atomicAdd(hist + kBuckets + b, static_cast<uint32_t>(ui & 0xFFFFFull));
+        for (int e0 = 0; e0 < words; e0 += 4) {
+            float s[4];
+            double u[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) s[q] = score((e0 + q) * 32 + lane);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) u[q] = mass_of(s[q], smax);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                U += u[q];
+                if (u[q] > 0.0) hist_add(hist, ykey(s[q], smax, g) >> 16, u[q]);
             }
-            U += u;
         }
         U = warp_sum(U);
-        __syncwarp();
         const double thr = static_cast<double>(prm.p) * U;
+        __syncwarp();
 
-        // bucket B* holding the last kept block, and the mass before it
-        double hm[kBuckets / 32], tot = 0.0;
+        // refine: at level L the cell is the blocks whose key has the L bytes
+        // fixed so far; its bins are the key's next byte
+        double before = 0.0;  // mass ranked above the cell
+        uint32_t prefix = 0;  // key bytes fixed so far
+        bool done = false;
+        for (int lvl = 0; lvl < 3 && !done; ++lvl) {
+            const int pshift = 24 - 8 * lvl, dshift = 16 - 8 * lvl;
+            // scan of the cell's bins (8 per lane, in rank order)
+            double hm[8], tot = 0.0;
 #pragma unroll
-        for (int k = 0; k < kBuckets / 32; ++k) {
-            const int b = lane * (kBuckets / 32) + k;
-            hm[k] = static_cast<double>(hist[b]) * 1048576.0 + static_cast<double>(hist[kBuckets + b]);
-            tot += hm[k];
-        }
-        double incl = tot;
+            for (int k = 0; k < 8; ++k) {
+                const int b = lane * 8 + k;
+                hm[k] = static_cast<double>(hist[b]) * 1048576.0 + static_cast<double>(hist[256 + b]);
+                tot += hm[k];
+            }
+            double incl = tot;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const double v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-        }
-        const unsigned crossing = __ballot_sync(0xffffffffu, incl >= thr);
-        int bstar = kBuckets;  // no crossing only for a non-finite row: keep it whole
-        double before = 0.0;
-        if (crossing != 0u) {
+            for (int o = 1; o < 32; o <<= 1) {
+                const double v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const unsigned crossing = __ballot_sync(0xffffffffu, before + incl >= thr);
+            if (crossing == 0u) {  // only a row with non-finite scores: keep it whole
+                for (int e = lane; e < words; e += 32) sw[e] = 0xFFFFFFFFu;
+                done = true;
+                break;
+            }
             const int owner = __ffs(crossing) - 1;
             int kk = 0;
-            double c = incl - tot;
+            double c = before + incl - tot;
 #pragma unroll
-            for (int k = 0; k < kBuckets / 32; ++k) {
+            for (int k = 0; k < 8; ++k) {
                 if (c + hm[k] >= thr) break;
                 c += hm[k];
                 ++kk;
             }
-            bstar = __shfl_sync(0xffffffffu, lane * (kBuckets / 32) + kk, owner);
+            const uint32_t dig = static_cast<uint32_t>(__shfl_sync(0xffffffffu, lane * 8 + kk, owner));
             before = __shfl_sync(0xffffffffu, c, owner);
-        }
-        __syncwarp();  // histogram read by all lanes before the entries overwrite it
-
-        // exact rank of the last kept block inside bucket B*: the largest rank
-        // key c with before + mass(B* blocks ranked at or above c) >= thr
-        uint64_t kstar = 0;
-        if (bstar < kBuckets) {
-            int m = 0;
-            uint64_t kx = 0, kfirst = 0;
-            bool have_first = false;
-            for (int e = 0; e < words; ++e) {
-                const int j = e * 32 + lane;
-                bool in = false;
-                double u = 0.0;
-                float s = 0.f;
-                if (j < nb) {
-                    s = srow[j];
-                    if (bucket_of(s, smax) == bstar) {
-                        u = mass_of(s, smax);
-                        in = u > 0.0;
-                    }
-                }
-                const unsigned bal = __ballot_sync(0xffffffffu, in);
-                if (bal == 0u) continue;
-                if (in) {
-                    const int pos = m + __popc(bal & lt);
-                    if (pos < kListCap)
-                        ent[pos] = (static_cast<unsigned long long>(u) << 11) |
-                                   static_cast<unsigned long long>(j);
-                }
-                // common high bits of the bucket's rank keys narrow the search
-                const int src = __ffs(bal) - 1;
-                const uint64_t k0 = __shfl_sync(0xffffffffu, in ? rank_key(s, j) : 0ull, src);
-                if (!have_first) {
-                    kfirst = k0;
-                    have_first = true;
-                }
-                if (in) kx |= rank_key(s, j) ^ kfirst;
-                m += __popc(bal);
-            }
+            __syncwarp();  // every lane has read the bins
+            const bool refine = lvl < 2;
+            if (refine) clear_hist();
             __syncwarp();
+
+            // one pass: cell blocks in lower bins are kept; those in the
+            // crossing bin are the candidates (the first 64 listed) and, for
+            // the next level, histogrammed by the next byte
+            const int nshift = dshift - 8;
+            int m = 0;
+            for (int e0 = 0; e0 < words; e0 += 4) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) kx |= __shfl_xor_sync(0xffffffffu, kx, o);
-            const int top = kx ? 63 - __clzll(static_cast<long long>(kx)) : -1;
-            // mass of bucket B*'s blocks with rank key >= c (exact sum)
-            auto mass_ge = [&](uint64_t c) -> double {
-                double a = 0.0;
-                if (m <= kListCap) {
-                    for (int k = lane; k < m; k += 32) {
-                        const unsigned long long v = ent[k];
-                        const int j = static_cast<int>(v & 0x7FFull);
-                        if (rank_key(srow[j], j) >= c) a += static_cast<double>(v >> 11);
-                    }
-                } else {  // a bucket too full for the scratch: recompute its masses
-                    for (int j = lane; j < nb; j += 32) {
-                        const float s = srow[j];
-                        if (bucket_of(s, smax) == bstar && rank_key(s, j) >= c)
-                            a += mass_of(s, smax);
+                for (int q = 0; q < 4; ++q) {
+                    const int e = e0 + q;
+                    if (e < words) {
+                        const float s = score(e * 32 + lane);
+                        const uint32_t y = ykey(s, smax, g);
+                        const bool member = s > -INFINITY && (lvl == 0 || (y >> pshift) == prefix);
+                        const uint32_t b = (y >> dshift) & 255u;
+                        const unsigned above = __ballot_sync(0xffffffffu, member && b < dig);
+                        const bool cand = member && b == dig;
+                        const unsigned bc = __ballot_sync(0xffffffffu, cand);
+                        if (lane == 0) sw[e] = lvl == 0 ? above : (sw[e] | above);
+                        if (cand) {
+                            const int pos = m + __popc(bc & lt);
+                            if (pos < kCand) ent[pos] = e * 32 + lane;
+                            if (refine) {
+                                const double u = mass_of(s, smax);
+                                if (u > 0.0) hist_add(hist, (y >> nshift) & 255u, u);
+                            }
+                        }
+                        m += __popc(bc);
                     }
                 }
-                return warp_sum(a);
-            };
-            // invariant: before + mass_ge(kstar) >= thr (the whole bucket reaches it)
-            kstar = top >= 0 ? (kfirst & ~((2ull << top) - 1ull)) : kfirst;
-            for (int b = top; b >= 0; --b) {
-                const uint64_t cand = kstar | (1ull << b);
-                if (before + mass_ge(cand) >= thr) kstar = cand;
+            }
+            prefix = (prefix << 8) | dig;
+            __syncwarp();
+            if (m <= kCand) {
+                // exact rank among the candidates: the last kept block is the
+                // highest-ranked candidate whose inclusive mass (candidates
+                // ranked at or above it) reaches thr - before
+                int jc[2];
+                double uc[2];
+                uint64_t Kc[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int slot = h * 32 + lane;
+                    jc[h] = slot < m ? ent[slot] : 0;
+                    const float s = slot < m ? srow[jc[h]] : -INFINITY;
+                    uc[h] = slot < m ? mass_of(s, smax) : 0.0;
+                    Kc[h] = slot < m ? rank_key(s, jc[h]) : 0ull;
+                }
+                double S[2] = {0.0, 0.0};
+                for (int t = 0; t < m; ++t) {
+                    const uint64_t Kt = __shfl_sync(0xffffffffu, t < 32 ? Kc[0] : Kc[1], t & 31);
+                    const double ut = __shfl_sync(0xffffffffu, t < 32 ? uc[0] : uc[1], t & 31);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        if (Kt >= Kc[h]) S[h] += ut;
+                }
+                uint64_t best = 0ull;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    if (h * 32 + lane < m && before + S[h] >= thr) best = max(best, Kc[h]);
+                const uint64_t kstar = warp_max_u64(best);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    if (h * 32 + lane < m && Kc[h] >= kstar)
+                        atomicOr(sw + (jc[h] >> 5), 1u << (jc[h] & 31));
+                done = true;
             }
         }
-
-        // bit row: adaptive set, then the STA window and the diagonal
-        for (int e = 0; e < words; ++e) {
-            const int j = e * 32 + lane;
-            bool keep = false;
-            if (j < nb) {
-                const float s = srow[j];
-                const int b = bucket_of(s, smax);
-                keep = b < bstar || (b == bstar && rank_key(s, j) >= kstar);
+        if (!done) {
+            // more than 64 blocks share all three key bytes: take the cell's
+            // score groups from the top (one score per group, so one mass);
+            // the group that reaches thr keeps its lowest indices first
+            uint64_t bound = 1ull << 32;  // groups at or above this order key are taken
+            for (int guard = 0; guard < nb; ++guard) {
+                uint32_t okm = 0u;
+                bool any = false;
+                for (int e = 0; e < words; ++e) {
+                    const float s = score(e * 32 + lane);
+                    const uint32_t ok = order_key(s);
+                    if (s > -INFINITY && ykey(s, smax, g) == prefix && ok < bound) {
+                        okm = max(okm, ok);
+                        any = true;
+                    }
+                }
+                if (__ballot_sync(0xffffffffu, any) == 0u) break;
+                const uint32_t tau = __reduce_max_sync(0xffffffffu, any ? okm : 0u);
+                // the group's score (order_key inverted) and its common mass
+                const float sg = __uint_as_float((tau & 0x80000000u) ? (tau & 0x7FFFFFFFu) : ~tau);
+                const double ug = mass_of(sg, smax);
+                int gn = 0;
+                for (int e = 0; e < words; ++e) {
+                    const float s = score(e * 32 + lane);
+                    gn += __popc(__ballot_sync(0xffffffffu, s > -INFINITY &&
+                                                                ykey(s, smax, g) == prefix &&
+                                                                order_key(s) == tau));
+                }
+                const bool last = before + static_cast<double>(gn) * ug >= thr;
+                int t = gn;  // members of the group kept, lowest index first
+                if (last) {
+                    t = static_cast<int>(ceil((thr - before) / ug));
+                    while (t > 1 && before + static_cast<double>(t - 1) * ug >= thr) --t;
+                    while (t < gn && before + static_cast<double>(t) * ug < thr) ++t;
+                }
+                int seen = 0;
+                for (int e = 0; e < words; ++e) {
+                    const float s = score(e * 32 + lane);
+                    const bool in = s > -INFINITY && ykey(s, smax, g) == prefix && order_key(s) == tau;
+                    const unsigned b = __ballot_sync(0xffffffffu, in);
+                    const unsigned kb = __ballot_sync(0xffffffffu, in && seen + __popc(b & lt) < t);
+                    if (lane == 0) sw[e] |= kb;
+                    seen += __popc(b);
+                }
+                before += static_cast<double>(gn) * ug;
+                if (last) break;
+                bound = tau;
             }
-            const unsigned bal = __ballot_sync(0xffffffffu, keep);
-            if (lane == 0) sw[e] = bal;
         }
         __syncwarp();
+
+        // the diagonal and the STA window
         if (lane == 0) atomicOr(sw + (i >> 5), 1u << (i & 31));
         if (!(prm.flags & 1u)) {
             // the window clipped to the grid, enumerated block by block
@@ -523,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             cnt += __popc(word);
         }
         if (lane == 0) row_cnt[bh * nb + i] = cnt;
-        __syncwarp();  // sw and the scratch are reused by the next row
+        __syncwarp();  // sw, the histogram and the list are reused by the next row
     }
 }
 
@@ -654,9 +730,9 @@ __global__ void __launch_bounds__(kColWarps * 32) col_lists_kernel(
 // ---------------------------------------------------------------------------
 size_t nabla_score_cut_smem(int nb, int D) {
     const size_t nbp = (static_cast<size_t>(nb) + 3) & ~static_cast<size_t>(3);
-    return sizeof(float) * (nabla::kRows * nbp + static_cast<size_t>(D) * nabla::kRows +
-                            nabla::kStages * nabla::kDc * nabla::kCols) +
-           sizeof(uint32_t) * nabla::kWarps * nabla::kMaxWords;
+    return sizeof(float) * (nabla::kRows * nbp + static_cast<size_t>(D) * nabla::kRows) +
+           sizeof(uint32_t) * nabla::kWarps * (nabla::kHistWords + nabla::kMaxWords) +
+           sizeof(int) * nabla::kWarps * nabla::kCand;
 }
 
 template <int D>
