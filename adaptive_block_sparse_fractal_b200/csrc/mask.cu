@@ -22,6 +22,7 @@
 // The mass sums are exact integers, so the selected set does not depend on
 // the order in which threads add them.
 #include "common.cuh"
+#include "exp_nonpos.cuh"
 
 namespace nabla {
 
@@ -193,10 +194,11 @@ __global__ void __launch_bounds__(256) flatten_pool_kernel(
 constexpr int kRows = 16;       // query blocks per CTA
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kHistWords = 512;     // per warp: 256 bins x (hi, lo) u32
+constexpr int kBins = 256;          // bins of one row's mass histogram
+constexpr int kHistWords = 2 * kBins;  // per warp: hi and lo u32 sums per bin
 constexpr int kMaxWords = 64;       // bit-row words of the largest row (2048 blocks)
 constexpr int kCand = 64;           // candidates ranked exactly by one warp at once
-constexpr int kPre = 16;            // features of K-bar prefetched ahead in registers
+constexpr int kPre = 8;             // features of K-bar prefetched ahead in registers
 
 struct CutParams {
     int nb, T, Hp, Wp, wt, wh, ww;
@@ -220,7 +222,7 @@ __device__ __forceinline__ uint64_t rank_key(float s, int j) {
 // integer <= 2^40; sums of up to 2^12 of them stay below 2^53, so every sum
 // below is exact whatever the order of the additions).  s = -inf gives 0.
 __device__ __forceinline__ double mass_of(float s, float smax) {
-    const double w = exp(static_cast<double>(s) - static_cast<double>(smax));
+    const double w = exp_nonpos(static_cast<double>(s) - static_cast<double>(smax));
     return trunc(w * 1099511627776.0);  // * 2^40 is an exact scaling
 }
 
@@ -248,19 +250,23 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t v) {
     return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
+// Bin b holds hi = sum (u >> 20) and lo = sum (u & (2^20 - 1)); with masses
+// u <= 2^40 each stays below 2^31 for up to 2048 blocks, so the u32 sums are
+// exact (and cheaper than 64-bit shared atomics).
 __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t b, double u) {
     const unsigned long long ui = static_cast<unsigned long long>(u);
     atomicAdd(hist + b, static_cast<uint32_t>(ui >> 20));
-    atomicAdd(hist + 256 + b, static_cast<uint32_t>(ui & 0xFFFFFull));
+    atomicAdd(hist + kBins + b, static_cast<uint32_t>(ui & 0xFFFFFull));
 }
 
 // One CTA per (bh, 16 query blocks).
 //   Phase 1: the 16 x nb pooled scores into shared memory.  Thread t owns
-//            columns t, t + 256, ...; for each it runs the 16 rows' fma chains
-//            over d = 0 .. D-1 as packed fma.rn.f32x2 on row pairs (each lane
-//            rounds like fmaf), the query means broadcast from shared memory
-//            and the K-bar^T column read from L2 with 16 features prefetched
-//            in registers; then times scale.
+//            the column pairs (2t, 2t + 1), (2t + 512, 2t + 513), ...; for each
+//            it runs the 32 fma chains (16 rows x 2 columns) over d = 0 .. D-1
+//            as packed fma.rn.f32x2 on row pairs (each lane rounds like fmaf),
+//            the query means broadcast from shared memory and the K-bar^T
+//            column pair read from L2 with 8 features prefetched in registers;
+//            then times scale.
 //   Phase 2: one warp per row.  Exact integer masses are summed into a
 //            256-bin histogram over the top byte of the bucket key (bins
 //            spread over the row's own score range); its scan gives the bin
@@ -300,29 +306,37 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     const float *kt = kbar_t + bh * static_cast<int64_t>(D) * nbp;
     const uint64_t sc2 = f2_pack(prm.scale, prm.scale);
-    for (int j = tid; j < nb; j += kThreads) {
-        uint64_t acc[kRows / 2];
+    for (int pc = tid; 2 * pc < nbp; pc += kThreads) {
+        const int j = 2 * pc;  // columns j, j + 1 (pad columns past nb are zero)
+        uint64_t acc[2][kRows / 2];
 #pragma unroll
-        for (int q = 0; q < kRows / 2; ++q) acc[q] = 0ull;
-        float kc[kPre], kn[kPre];
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-        for (int q = 0; q < kPre; ++q) kc[q] = __ldg(kt + static_cast<int64_t>(q) * nbp + j);
+            for (int q = 0; q < kRows / 2; ++q) acc[c][q] = 0ull;
+        float2 kc[kPre], kn[kPre];
+#pragma unroll
+        for (int q = 0; q < kPre; ++q)
+            kc[q] = __ldg(reinterpret_cast<const float2 *>(kt + static_cast<int64_t>(q) * nbp + j));
 #pragma unroll
         for (int d0 = 0; d0 < D; d0 += kPre) {
             if (d0 + kPre < D) {
 #pragma unroll
                 for (int q = 0; q < kPre; ++q)
-                    kn[q] = __ldg(kt + static_cast<int64_t>(d0 + kPre + q) * nbp + j);
+                    kn[q] = __ldg(reinterpret_cast<const float2 *>(
+                        kt + static_cast<int64_t>(d0 + kPre + q) * nbp + j));
             }
 #pragma unroll
             for (int q = 0; q < kPre; ++q) {
                 const float4 *qv = reinterpret_cast<const float4 *>(sQt + (d0 + q) * kRows);
-                const uint64_t kk = f2_pack(kc[q], kc[q]);
+                const uint64_t k0 = f2_pack(kc[q].x, kc[q].x), k1 = f2_pack(kc[q].y, kc[q].y);
 #pragma unroll
                 for (int v = 0; v < kRows / 4; ++v) {
                     const float4 qq = qv[v];
-                    acc[2 * v] = f2_fma(f2_pack(qq.x, qq.y), kk, acc[2 * v]);
-                    acc[2 * v + 1] = f2_fma(f2_pack(qq.z, qq.w), kk, acc[2 * v + 1]);
+                    const uint64_t qa = f2_pack(qq.x, qq.y), qb = f2_pack(qq.z, qq.w);
+                    acc[0][2 * v] = f2_fma(qa, k0, acc[0][2 * v]);
+                    acc[0][2 * v + 1] = f2_fma(qb, k0, acc[0][2 * v + 1]);
+                    acc[1][2 * v] = f2_fma(qa, k1, acc[1][2 * v]);
+                    acc[1][2 * v + 1] = f2_fma(qb, k1, acc[1][2 * v + 1]);
                 }
             }
             if (d0 + kPre < D) {
@@ -332,9 +346,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
 #pragma unroll
         for (int q = 0; q < kRows / 2; ++q) {
-            const uint64_t a = f2_mul(acc[q], sc2);
-            sS[(2 * q) * nbp + j] = f2_lo(a);
-            sS[(2 * q + 1) * nbp + j] = f2_hi(a);
+            const uint64_t a = f2_mul(acc[0][q], sc2), b = f2_mul(acc[1][q], sc2);
+            *reinterpret_cast<float2 *>(sS + (2 * q) * nbp + j) = make_float2(f2_lo(a), f2_lo(b));
+            *reinterpret_cast<float2 *>(sS + (2 * q + 1) * nbp + j) = make_float2(f2_hi(a), f2_hi(b));
         }
     }
     __syncthreads();  // scores complete
@@ -389,20 +403,19 @@ __global__ void __launch_bounds__(kThreads, 2)
         const float g = __fdiv_rn(256.0f, span);
 
         // level 0: every block's mass into the bin of its key's top byte, and
-        // the row total.  The bins hold hi = sum (u >> 20) and lo = sum (u &
-        // (2^20 - 1)); each stays below 2^31 for up to 2048 blocks (exact).
+        // the row total
         clear_hist();
         __syncwarp();
         double U = 0.0;
-        for (int e0 = 0; e0 < words; e0 += 4) {
-            float s[4];
-            double u[4];
+        for (int e0 = 0; e0 < words; e0 += 8) {
+            float s[8];
+            double u[8];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) s[q] = score((e0 + q) * 32 + lane);
+            for (int q = 0; q < 8; ++q) s[q] = score((e0 + q) * 32 + lane);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) u[q] = mass_of(s[q], smax);
+            for (int q = 0; q < 8; ++q) u[q] = mass_of(s[q], smax);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 8; ++q) {
                 U += u[q];
                 if (u[q] > 0.0) hist_add(hist, ykey(s[q], smax, g) >> 16, u[q]);
             }
@@ -423,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int b = lane * 8 + k;
-                hm[k] = static_cast<double>(hist[b]) * 1048576.0 + static_cast<double>(hist[256 + b]);
+                hm[k] = static_cast<double>(hist[b]) * 1048576.0 + static_cast<double>(hist[kBins + b]);
                 tot += hm[k];
             }
             double incl = tot;
@@ -450,14 +463,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             const uint32_t dig = static_cast<uint32_t>(__shfl_sync(0xffffffffu, lane * 8 + kk, owner));
             before = __shfl_sync(0xffffffffu, c, owner);
             __syncwarp();  // every lane has read the bins
-            const bool refine = lvl < 2;
-            if (refine) clear_hist();
-            __syncwarp();
 
             // one pass: cell blocks in lower bins are kept; those in the
-            // crossing bin are the candidates (the first 64 listed) and, for
-            // the next level, histogrammed by the next byte
-            const int nshift = dshift - 8;
+            // crossing bin are the candidates (the first 64 listed)
             int m = 0;
             for (int e0 = 0; e0 < words; e0 += 4) {
 #pragma unroll
@@ -475,12 +483,23 @@ __global__ void __launch_bounds__(kThreads, 2)
                         if (cand) {
                             const int pos = m + __popc(bc & lt);
                             if (pos < kCand) ent[pos] = e * 32 + lane;
-                            if (refine) {
-                                const double u = mass_of(s, smax);
-                                if (u > 0.0) hist_add(hist, (y >> nshift) & 255u, u);
-                            }
                         }
                         m += __popc(bc);
+                    }
+                }
+            }
+            if (m > kCand && lvl < 2) {
+                // too many to rank at once: histogram the crossing bin's blocks
+                // by the key's next byte for the next level
+                const uint32_t cell = (prefix << 8) | dig;
+                clear_hist();
+                __syncwarp();
+                for (int e = 0; e < words; ++e) {
+                    const float s = score(e * 32 + lane);
+                    const uint32_t y = ykey(s, smax, g);
+                    if (s > -INFINITY && (y >> dshift) == cell) {
+                        const double u = mass_of(s, smax);
+                        if (u > 0.0) hist_add(hist, (y >> (dshift - 8)) & 255u, u);
                     }
                 }
             }
