@@ -37,13 +37,42 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch, per
-# head, from one ncu capture of `bench.py --heads 8 --no-sweep` (same shape,
-# 8 heads; heads are independent, so the traffic scales with their number).
-# Must be re-measured whenever these kernels change.
-NCU_DRAM_BYTES_PER_HEAD = {
-    ("train", "attn_bwd"): (320.8e6 + 951.1e6 + 788.5e6) / 8,  # pre + dK/dV + dQ
-    ("train", "attn_fwd"): (475.9e6 + 144.8e6) / 8,
+# head, from one ncu capture of `bench.py --heads 8` (same shape, 8 heads;
+# heads are independent, so the traffic scales with their number), with the
+# SHA-256 (first 12 hex digits) of the kernel sources it was taken from.  When
+# the sources no longer match, the bench reports no traffic rather than a
+# stale figure.
+NCU_DRAM = {
+    # pre 317.0 + 3.7 MB, dK/dV 661.1 + 292.1 MB, dQ 646.4 + 141.9 MB at 8 heads
+    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.65e6 + 661.14e6 + 292.06e6
+                                               + 646.42e6 + 141.87e6) / 8,
+                            "sources_sha": "5a197c27ba01"},
+    # 475.2 + 145.5 MB at 8 heads
+    ("train", "attn_fwd"): {"bytes_per_head": (475.19e6 + 145.54e6) / 8,
+                            "sources_sha": "b3658f1cf267"},
 }
+KERNEL_SOURCES = {
+    "attn_bwd": ("attn_bwd_sm100.cu", "sm100.cuh", "common.cuh"),
+    "attn_fwd": ("attn_fwd_sm100.cu", "sm100.cuh", "common.cuh"),
+}
+# dense bf16 tensor-core work of one SM per clock: two M=128 x N=128 x K=128
+# MMAs (2 x 4.19 MFLOP) take 1024 cycles
+TENSOR_FLOP_PER_CLK_SM = 8192
+NUM_SMS = 148
+
+
+def sources_sha(op):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[op]:
+        with open(os.path.join(ROOT, "adaptive_block_sparse_fractal_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def tensor_peak_at_clock(sm_mhz):
+    """TFLOP/s of the tensor pipes of all SMs at the given SM clock."""
+    return NUM_SMS * TENSOR_FLOP_PER_CLK_SM * sm_mhz * 1e6 / 1e12 if sm_mhz else None
 
 
 def parse(argv=None):
@@ -157,33 +186,70 @@ class Clocks:
 # --------------------------------------------------------------------------
 # CPU oracle timing (bounded sample)
 # --------------------------------------------------------------------------
-def oracle_sample(w, n_blocks=24, seed=0):
-    """Oracle on one head of the workload: its mask (all rows) and the forward
-    on n_blocks sampled query blocks.  Returns (kept fwd FLOP, fwd seconds,
-    mask seconds, cores, description)."""
+def oracle_sample(w, n_fwd=8, n_dq=4, seed=0):
+    """The oracle on a bounded sample of one head of the workload, timed, and
+    extrapolated to one whole step (all heads, mask + forward + backward).
+
+    Timed: the mask of the head (every row), the forward of n_fwd sampled query
+    blocks, and the backward of n_dq sampled query blocks (dQ) plus one key
+    block (dK, dV).  The oracle's backward recomputes the
+    forward rows it needs (LSE and D of every query block the selection
+    touches), so its FLOPs are counted as it performs them.  The key block is
+    the one with the shortest column list of the head, which bounds the rows
+    it needs; the rates measured are per FLOP, so the choice does not bias
+    the extrapolation:
+      forward      4 * 64 * 64 * D per kept block pair of a selected row,
+      LSE rows     4 * 64 * 64 * D per kept pair of every needed query block,
+      dQ           6 * 64 * 64 * D per kept pair (S, dP, dQ),
+      dK, dV       8 * 64 * 64 * D per kept pair of the column (S, dP, dV, dK).
+    A whole step in the oracle is then, per head, the mask plus every kept
+    pair at 4 (forward) + 18 (backward: LSE rows, dQ loop, dK/dV loop) units,
+    each part at the rate measured on its sample.  Returns a dict with the
+    extrapolated seconds per step, the step's kept-pair FLOP count (the metric's
+    14 units per pair, as on the GPU) and a description."""
     import numpy as np
     import oracle
     from adaptive_block_sparse_fractal_b200 import synth
     w1 = synth.Workload(w.name, 1, 1, w.T, w.H, w.W, w.D, w.cell, w.p, w.window)
-    inp = synth.make_inputs(w1, seed, with_dout=False)
+    inp = synth.make_inputs(w1, seed, with_dout=True)
     flat = {n: oracle.flatten_tokens(synth.bits(inp[n]).reshape(1, w.N, w.D), w.T, w.H, w.W, w.P)
             for n in ("q", "k", "v")}
+    dout = synth.bits(inp["dout"]).reshape(1, w.N, w.D)
     t0 = time.perf_counter()
-    m = oracle.build_mask(flat["q"], flat["k"], w.grid_blocks, w.p, w.scale, w.window, cols=False)
+    m = oracle.build_mask(flat["q"], flat["k"], w.grid_blocks, w.p, w.scale, w.window, cols=True)
     t_mask = time.perf_counter() - t0
-    rng = np.random.default_rng(seed)
-    sel = [(0, int(i)) for i in rng.choice(w.nb, n_blocks, replace=False)]
     q, k, v = (oracle.bf16_bits_to_f64(flat[n]) for n in ("q", "k", "v"))
+    do = oracle.bf16_bits_to_f64(dout)
+    rc, cc = m["row_cnt"][0], m["col_cnt"][0]
+    unit = 64.0 * 64 * w.D
+    rng = np.random.default_rng(seed)
+    fsel = [int(i) for i in rng.choice(w.nb, n_fwd, replace=False)]
     t0 = time.perf_counter()
-    oracle.attn_fwd(q, k, v, m["row_idx"], m["row_cnt"], w.scale, sel=sel)
+    oracle.attn_fwd(q, k, v, m["row_idx"], m["row_cnt"], w.scale, sel=[(0, i) for i in fsel])
     t_fwd = time.perf_counter() - t0
-    kept = sum(int(m["row_cnt"][0, i]) for _, i in sel)
-    flop = 4.0 * 64 * 64 * w.D * kept
+    rate_fwd = 4 * unit * float(rc[fsel].sum()) / t_fwd
+    qsel = [int(i) for i in rng.choice(w.nb, n_dq, replace=False)]
+    kj = int(np.argmin(cc))
+    need = set(qsel) | set(int(i) for i in m["col_idx"][0, kj, :cc[kj]])
+    bwd_flop = unit * (4 * float(sum(int(rc[i]) for i in need)) + 6 * float(rc[qsel].sum())
+                       + 8 * float(cc[kj]))
+    t0 = time.perf_counter()
+    oracle.attn_bwd(q, k, v, do, m["row_idx"], m["row_cnt"], m["col_idx"], m["col_cnt"],
+                    w.scale, dq_sel=[(0, i) for i in qsel], kv_sel=[(0, kj)])
+    t_bwd = time.perf_counter() - t0
+    rate_bwd = bwd_flop / t_bwd
+    kept_head = float(rc.sum())
+    s_step = w.BH * (t_mask + kept_head * (4 * unit / rate_fwd + 18 * unit / rate_bwd))
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    desc = ("oracle (float64 C, OpenMP) on one head of the same workload: mask build for all "
-            "%d rows (%.2f s) + forward on %d sampled query blocks (%d kept block pairs); value "
-            "= kept forward FLOP / forward seconds" % (w.nb, t_mask, n_blocks, kept))
-    return flop, t_fwd, t_mask, cores, desc
+    desc = ("oracle (float64 C, OpenMP, %d threads) on one head of the same workload: mask for all "
+            "%d rows (%.2f s), forward of %d sampled query blocks (%.2f s, %.1f GFLOP/s), backward "
+            "of %d sampled query blocks + 1 key block with the forward rows it recomputes "
+            "(%d query blocks; %.2f s, %.1f GFLOP/s); extrapolated to %d heads x all %d kept "
+            "pairs per head: %.0f s per step" % (cores, w.nb, t_mask, n_fwd, t_fwd, rate_fwd / 1e9,
+                                                 n_dq, len(need), t_bwd, rate_bwd / 1e9, w.BH,
+                                                 int(kept_head), s_step))
+    return {"s_step": s_step, "flop_step": 14 * unit * kept_head * w.BH, "cores": cores,
+            "desc": desc, "sample_s": t_mask + t_fwd + t_bwd}
 
 
 # --------------------------------------------------------------------------
@@ -261,28 +327,90 @@ def long_p_sweep(dev, reps=5, warmup=3):
             "rows": rows}
 
 
+def config_timings(dev, reps=20, warmup=5):
+    """The two small workloads, each call timed on its own with CUDA events
+    (median of `reps` after `warmup`), with a 256 MB write between repetitions
+    so that every timed call starts from a cold L2 (their inputs fit in it):
+      tiny   (2 heads, 4 x 16 x 16, D = 64, p = 0.9): flatten of Q, mask build
+             from the flattened Q and K, forward;
+      small  (24 heads, 8 x 32 x 32, D = 128, p = 0.8): mask build, forward."""
+    import statistics as st
+    import torch
+    from adaptive_block_sparse_fractal_b200 import nabla, synth
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        out = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            b.synchronize()
+            out.append(a.elapsed_time(b))
+        return st.median(out)
+
+    res = {}
+    for name in ("tiny", "small"):
+        w = synth.WORKLOADS[name]
+        shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
+        prm = nabla.params_of(w.p, w.window, D=w.D)
+        grid = synth.make_inputs_device(w, 0, dev, with_dout=False)
+        q, k, v = (nabla.flatten(grid[n], w.T, w.H, w.W, w.P) for n in ("q", "k", "v"))
+        mask = nabla.alloc_mask(shape, dev, cols=False)
+        ws_m = nabla.workspace(shape, nabla.OP_BUILD_MASK, dev)
+        ws_f = nabla.workspace(shape, nabla.OP_ATTN_FWD, dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.BH, w.N), dtype=torch.float32, device=dev)
+        fq = torch.empty_like(q)
+        row = {"workload": "%s: B=%d heads=%d T*H*W=%dx%dx%d (%d tokens, %d blocks) D=%d p=%.2f "
+                           "STA %dx%dx%d" % (name, w.B, w.heads, w.T, w.H, w.W, w.N, w.nb, w.D, w.p,
+                                             *w.window),
+               "l2": "256 MB write before every timed call"}
+        if name == "tiny":
+            t = timed(lambda: nabla.flatten(grid["q"], w.T, w.H, w.W, w.P, out=fq))
+            row["flatten_ms"] = t
+            row["flatten_gbs"] = 2.0 * q.numel() * 2 / (t * 1e-3) / 1e9
+        t_mask = timed(lambda: nabla.build_mask(shape, prm, q, k, mask=mask, ws=ws_m))
+        t_fwd = timed(lambda: nabla.attn_fwd(shape, prm, q, k, v, mask, o=o, lse=lse, ws=ws_f))
+        kept = int(mask["row_cnt"].sum().item())
+        mask_bytes = 4.0 * w.N * w.D * w.BH + 16.0 * w.nb * w.D * w.BH + w.nb * w.nb * w.BH / 8.0 \
+            + 2.0 * kept + 4.0 * w.BH * w.nb
+        row.update({"build_mask_ms": t_mask, "build_mask_gbs": mask_bytes / (t_mask * 1e-3) / 1e9,
+                    "attn_fwd_ms": t_fwd, "kept_fraction": kept / (w.BH * w.nb * w.nb),
+                    "attn_fwd_tflops": 4.0 * 64 * 64 * w.D * kept / (t_fwd * 1e-3) / 1e12})
+        res[name] = row
+        del grid, q, k, v, mask, ws_m, ws_f, o, lse, fq
+    del flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_reference(args):
     rank, world, _ = dist_init(args.gpus)
     if rank != 0:
         return 0
     w = workload_of(args)
-    times, flops = [], []
+    steps = []
     for s in range(args.warmup + args.steps):
-        t0 = time.perf_counter()
-        flop, t_fwd, t_mask, cores, desc = oracle_sample(w, n_blocks=8, seed=s)
-        dt = time.perf_counter() - t0
+        r = oracle_sample(w, seed=s)
         if s >= args.warmup:
-            times.append(t_fwd)
-            flops.append(flop)
-    value = sum(flops) / sum(times) / 1e12
+            steps.append(r)
+    s_step = sum(r["s_step"] for r in steps) / len(steps)
+    value = sum(r["flop_step"] for r in steps) / sum(r["s_step"] for r in steps) / 1e12
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": workload_config(w),
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": desc.replace("24 sampled", "8 sampled")},
+        "ms_per_step": 1e3 * s_step, "ms_per_step_kind": "extrapolated from a timed sample",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": steps[-1]["cores"],
+                         "kind": "oracle", "sample": steps[-1]["desc"],
+                         "extrapolated_ms_per_step": 1e3 * s_step},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -391,15 +519,25 @@ def run_nabla(args):
     dom = max(ops, key=lambda k: ops[k][0])
     achieved = ops[dom][1] / (ops[dom][0] * 1e-3) / 1e12
     peak = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    traffic = None
-    per_head = NCU_DRAM_BYTES_PER_HEAD.get((args.workload, dom))
-    if per_head is not None:
-        traffic = per_head * w.heads
+    traffic, traffic_note = None, "no ncu capture recorded for this kernel"
+    cap = NCU_DRAM.get((args.workload, dom))
+    if cap is not None and cap["bytes_per_head"] is not None:
+        if cap["sources_sha"] == sources_sha(dom):
+            traffic = cap["bytes_per_head"] * w.heads
+            traffic_note = ("ncu capture of bench.py --heads 8 (kernel sources %s), scaled to %d "
+                            "heads" % (cap["sources_sha"], w.heads))
+        else:
+            traffic_note = "stale: the kernel sources changed since the ncu capture"
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": traffic, "kernel": dom,
-                "peak_source": "bf16 sustained (of %s)" % pk_src,
+                "frac": achieved / peak, "traffic": traffic, "traffic_note": traffic_note,
+                "kernel": dom, "peak_source": "bf16 sustained (of %s)" % pk_src,
                 "flop_per_launch": ops[dom][1], "ms_per_launch": ops[dom][0],
                 "frac_of_burst": achieved / pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])}
+    clk_peak = tensor_peak_at_clock(clk.get("sm_mhz"))
+    if clk_peak:
+        # the same work against the tensor pipes' own rate at this run's clock
+        roofline["frac_at_clock"] = achieved / clk_peak
+        roofline["peak_at_clock"] = clk_peak
 
     # ---- end to end through the C ABI with host buffers (pinned).  Every step
     # uploads its inputs from pinned host memory and downloads its results;
@@ -472,17 +610,19 @@ def run_nabla(args):
                          "neighbouring steps' compute"}
         del dev_in, dev_out
 
-    sweep = None
+    sweep, small_cfgs = None, None
     if rank == 0 and world == 1 and not args.no_sweep:
         B.clear()  # free this workload's buffers first
         torch.cuda.empty_cache()
         sweep = long_p_sweep(dev)
+        small_cfgs = config_timings(dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        flop, t_fwd, t_mask, cores, desc = oracle_sample(w)
-        cpu = {"value": flop / t_fwd / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": desc}
+        r = oracle_sample(w)
+        cpu = {"value": r["flop_step"] / r["s_step"] / 1e12, "unit": "TFLOP/s",
+               "cores": r["cores"], "kind": "oracle", "sample": r["desc"],
+               "extrapolated_ms_per_step": 1e3 * r["s_step"]}
 
     if rank == 0:
         line = {
@@ -498,11 +638,15 @@ def run_nabla(args):
             "kept_blocks": kept, "kept_fraction": kept_frac,
             "attn_fwd_tflops": fwd_flop / (phase[2] * 1e-3) / 1e12,
             "attn_bwd_tflops": bwd_flop / (phase[3] * 1e-3) / 1e12,
+            "attn_fwd_frac_at_clock": (fwd_flop / (phase[2] * 1e-3) / 1e12 / clk_peak
+                                       if clk_peak else None),
+            "attn_bwd_frac_at_clock": (bwd_flop / (phase[3] * 1e-3) / 1e12 / clk_peak
+                                       if clk_peak else None),
             "flatten_qk_build_mask_gbs": mask_gbs,
             "flatten_qk_build_mask_frac_hbm": mask_gbs / pk["hbm_gbs"],
             "flatten_v_gbs": flat_gbs,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
-            "long_p_sweep": sweep,
+            "long_p_sweep": sweep, "small_configs": small_cfgs,
             "gpu_launches": launches_per_step * args.steps,
         }
         print(json.dumps(line), flush=True)

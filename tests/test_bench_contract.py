@@ -18,6 +18,12 @@ def test_reference_arm_line_has_the_contract_keys(monkeypatch):
     monkeypatch.setenv("WORLD_SIZE", "1")
     monkeypatch.setenv("LOCAL_RANK", "0")
     args = bench.parse(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    # the arm's default workload is the 720p-like training step ...
+    assert bench.workload_of(args).N == 76800 and bench.workload_of(args).heads == 40
+    # ... whose oracle sample takes ~20 s of CPU; the line's keys are checked
+    # on the small workload's sample instead
+    from adaptive_block_sparse_fractal_b200 import synth
+    monkeypatch.setattr(bench, "workload_of", lambda a: synth.WORKLOADS["small"])
     buf = io.StringIO()
     with contextlib.redirect_stdout(buf):
         assert bench.run_reference(args) == 0
@@ -36,12 +42,15 @@ def test_reference_arm_line_has_the_contract_keys(monkeypatch):
     assert line["dtype"] == "f64" and line["data"] == "synthetic"
     # the same workload as the CUDA arm's line
     assert line["config"] == bench.workload_config(bench.workload_of(args))
-    assert "76800 tokens" in line["config"]["workload"]
+    assert line["ms_per_step_kind"] == "extrapolated from a timed sample"
 
     cb = line["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["unit"] == "TFLOP/s"
     assert cb["value"] == pytest.approx(line["value"])
     assert cb["cores"] >= 1 and "8 sampled query blocks" in cb["sample"]
+    assert "backward" in cb["sample"] and "extrapolated" in cb["sample"]
+    # the line's time is the extrapolated whole step, consistent with its value
+    assert cb["extrapolated_ms_per_step"] == pytest.approx(line["ms_per_step"])
 
     e2e = line["e2e"]
     assert e2e["value"] == pytest.approx(line["value"]) and e2e["unit"] == line["unit"]
