@@ -109,25 +109,37 @@ def bits(t: torch.Tensor):
 
 
 def make_inputs_device(w: Workload, seed0: int = 0, device="cuda", with_dout=None,
-                       rank: int = 0):
-    """Same recipe as make_inputs, drawn with a CUDA generator directly on the
-    device (fast for the benchmark's full-size workloads; the values differ
-    from the CPU stream).  Q, K, V in grid order [B*h, T*H*W, D], dout in
-    flattened order [B*h, N, D]; `rank` offsets the seeds."""
+                       head_range=None):
+    """Same recipe as make_inputs, drawn with a generator on `device` (fast for
+    the benchmark's full-size workloads; the values differ from the CPU
+    stream).  Every (batch, head) slice is drawn from its own seed, so any
+    subset of heads is the same as the corresponding slice of the whole
+    problem: `head_range` = (h0, h1) draws heads h0 .. h1 - 1 of every batch
+    element only (a partition of the heads over devices).  Q, K, V in grid
+    order [B*nh, T*H*W, D], dout in flattened order [B*nh, N, D], nh = h1 - h0."""
+    h0, h1 = (0, w.heads) if head_range is None else head_range
+    assert 0 <= h0 < h1 <= w.heads
     g = torch.Generator(device=device)
-    out = {}
     ct, cy, cx = w.cell
     nct, ncy, ncx = -(-w.T // ct), -(-w.H // cy), -(-w.W // cx)
+    sel = [b * w.heads + h for b in range(w.B) for h in range(h0, h1)]
+    out = {}
     for name, off in (("q", 1), ("k", 2), ("v", 3)):
-        g.manual_seed(int(seed0 + off + 1000 * rank))
-        c = torch.randn(w.BH, nct, ncy, ncx, w.D, generator=g, device=device)
-        c = (c.repeat_interleave(ct, 1).repeat_interleave(cy, 2).repeat_interleave(cx, 3)
-             [:, :w.T, :w.H, :w.W])
-        x = torch.randn(w.BH, w.T, w.H, w.W, w.D, generator=g, device=device)
-        x.mul_(w.noise).add_(c)
-        out[name] = x.to(torch.bfloat16).reshape(w.BH, w.N, w.D)
-        del c, x
+        x = torch.empty(len(sel), w.N, w.D, dtype=torch.bfloat16, device=device)
+        for n, bh in enumerate(sel):
+            g.manual_seed(int((seed0 + off) * 100003 + bh))
+            c = torch.randn(nct, ncy, ncx, w.D, generator=g, device=device)
+            c = (c.repeat_interleave(ct, 0).repeat_interleave(cy, 1).repeat_interleave(cx, 2)
+                 [:w.T, :w.H, :w.W])
+            t = torch.randn(w.T, w.H, w.W, w.D, generator=g, device=device)
+            t.mul_(w.noise).add_(c)
+            x[n] = t.to(torch.bfloat16).reshape(w.N, w.D)
+            del c, t
+        out[name] = x
     if with_dout or (with_dout is None and w.backward):
-        g.manual_seed(int(seed0 + 4 + 1000 * rank))
-        out["dout"] = torch.randn(w.BH, w.N, w.D, generator=g, device=device).to(torch.bfloat16)
+        x = torch.empty(len(sel), w.N, w.D, dtype=torch.bfloat16, device=device)
+        for n, bh in enumerate(sel):
+            g.manual_seed(int((seed0 + 4) * 100003 + bh))
+            x[n] = torch.randn(w.N, w.D, generator=g, device=device).to(torch.bfloat16)
+        out["dout"] = x
     return out

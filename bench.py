@@ -274,10 +274,31 @@ def max_over_ranks(x, world, device):
     return float(t.item())
 
 
-def whole_job_tflops(flop_per_rank, ms_per_step, world):
-    """Weak scaling: every rank runs the whole workload on its own batch, so
-    the job processes world x the per-rank FLOPs in the slowest rank's time."""
-    return world * flop_per_rank / (ms_per_step * 1e-3) / 1e12
+def head_range(heads, world, rank):
+    """Heads [h0, h1) of every batch element that rank `rank` of `world` owns:
+    the heads are split into equal contiguous runs, one per GPU (masks,
+    forward and backward are independent per head, so no data moves between
+    the GPUs)."""
+    if heads % world:
+        raise SystemExit("%d heads do not split evenly over %d GPUs" % (heads, world))
+    n = heads // world
+    return rank * n, (rank + 1) * n
+
+
+def sum_over_ranks(x, world, device):
+    """Sum of a per-rank scalar over all ranks (every rank gets it)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def whole_job_tflops(flop_all_ranks, ms_per_step):
+    """Strong scaling over a head partition: the job's FLOPs (all ranks'
+    heads of the one problem) in the slowest rank's time."""
+    return flop_all_ranks / (ms_per_step * 1e-3) / 1e12
 
 
 def long_p_sweep(dev, reps=5, warmup=3):
@@ -406,7 +427,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * s_step, "ms_per_step_kind": "extrapolated from a timed sample",
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": steps[-1]["cores"],
                          "kind": "oracle", "sample": steps[-1]["desc"],
@@ -429,11 +450,14 @@ def run_nabla(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     nabla.lib()
-    w = workload_of(args)
+    import dataclasses
+    w_job = workload_of(args)
+    h0, h1 = head_range(w_job.heads, world, rank)
+    w = dataclasses.replace(w_job, heads=h1 - h0)  # this rank's share of the problem
     shape = nabla.shape_of(w.B, w.heads, w.T, w.H, w.W, w.D, w.P)
     prm = nabla.params_of(w.p, w.window, D=w.D, flags=nabla.EMIT_COLS)
 
-    grid = synth.make_inputs_device(w, args.seed, dev, with_dout=True, rank=rank)
+    grid = synth.make_inputs_device(w_job, args.seed, dev, with_dout=True, head_range=(h0, h1))
     B = {
         "flat": {n: torch.empty_like(grid[n]) for n in ("q", "k", "v")},
         "o": torch.empty_like(grid["q"]),
@@ -478,7 +502,8 @@ def run_nabla(args):
         step(grid)
     barrier()
     kept = int(B["mask"]["row_cnt"].sum().item())
-    kept_frac = kept / (w.BH * w.nb * w.nb)
+    kept_all = sum_over_ranks(kept, world, dev)  # kept pairs of the whole problem
+    kept_frac = kept_all / (w_job.BH * w.nb * w.nb)
 
     # ---- device-resident timed region
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
@@ -503,9 +528,10 @@ def run_nabla(args):
     phase = [x / args.steps for x in phase]
     ms_step = total_ms / args.steps
 
-    fwd_flop = 4.0 * 64 * 64 * w.D * kept
+    fwd_flop = 4.0 * 64 * 64 * w.D * kept  # this rank's share
     bwd_flop = 10.0 * 64 * 64 * w.D * kept
-    value = whole_job_tflops(fwd_flop + bwd_flop, ms_step, world)
+    job_flop = 14.0 * 64 * 64 * w.D * kept_all
+    value = whole_job_tflops(job_flop, ms_step)
     N, D, BH, nb = w.N, w.D, w.BH, w.nb
     # flatten of Q and K (read grid, write flattened) + pooled means (write + read)
     # + bit rows + row and column lists
@@ -604,8 +630,9 @@ def run_nabla(args):
         e2e_ms = max_over_ranks(a.elapsed_time(b_), world, dev) / args.steps
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out.values())
-        e2e = {"value": whole_job_tflops(fwd_flop + bwd_flop, e2e_ms, world), "unit": "TFLOP/s",
-               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+        e2e = {"value": whole_job_tflops(job_flop, e2e_ms), "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d * world,
+               "d2h_bytes_per_step": d2h * world,
                "copies": "pinned host <-> device on a copy stream, overlapped with the "
                          "neighbouring steps' compute"}
         del dev_in, dev_out
@@ -628,14 +655,16 @@ def run_nabla(args):
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: seeded cell-correlated bf16 Q/K/V (cell 2x8x8, noise 0.5), dO ~ "
-                    "N(0,1); each rank its own batch",
-            "config": workload_config(w),
+                    "N(0,1), one seed per (batch, head)",
+            "config": dict(workload_config(w_job),
+                           parallelism="heads split over %d GPU(s), %d per GPU, no exchange"
+                                       % (world, w.heads)),
             "breakdown_ms": {"flatten_v": phase[0], "flatten_qk_build_mask": phase[1],
                              "attn_fwd": phase[2], "attn_bwd": phase[3],
                              "unflatten_out": phase[4]},
-            "kept_blocks": kept, "kept_fraction": kept_frac,
+            "kept_blocks": int(kept_all), "kept_fraction": kept_frac,
             "attn_fwd_tflops": fwd_flop / (phase[2] * 1e-3) / 1e12,
             "attn_bwd_tflops": bwd_flop / (phase[3] * 1e-3) / 1e12,
             "attn_fwd_frac_at_clock": (fwd_flop / (phase[2] * 1e-3) / 1e12 / clk_peak

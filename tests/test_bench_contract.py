@@ -37,7 +37,7 @@ def test_reference_arm_line_has_the_contract_keys(monkeypatch):
     assert (line["n_gpus"], line["steps"], line["warmup"]) == (1, 1, 3)
     assert line["ms_per_step"] > 0
     assert line["higher_is_better"] is True
-    assert line["scaling"] == "weak"
+    assert line["scaling"] == "strong"
     assert line["vs_baseline"] is None
     assert line["dtype"] == "f64" and line["data"] == "synthetic"
     # the same workload as the CUDA arm's line
