@@ -17,6 +17,12 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, in
                                     uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
                                     uint16_t *col_idx, int32_t *col_cnt, float *scores,
                                     cudaStream_t stream, const void *q_grid, const void *k_grid);
+cudaError_t nabla_launch_build_mask_dr(int64_t BH, int nb, int D, int T, int Hp, int Wp, int mode,
+                                       double gamma, double lambda, float tau, float scale, int wt,
+                                       int wh, int ww, unsigned flags, const void *q,
+                                       const void *k, float *qbar, float *kbar_t, uint32_t *bits,
+                                       uint16_t *row_idx, int32_t *row_cnt, uint16_t *col_idx,
+                                       int32_t *col_cnt, float *scores, cudaStream_t stream);
 cudaError_t nabla_launch_attn_fwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
                                       const void *k, const void *v, const uint16_t *row_idx,
                                       const int32_t *row_cnt, void *o, float *lse,
@@ -243,6 +249,44 @@ int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
         params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
         mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
         cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, q_grid, k_grid));
+}
+
+int nabla_build_mask_dr(const nabla_shape *shape, const nabla_dr_params *params,
+                        const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
+                        void *workspace, size_t workspace_bytes, nabla_stream_t stream) {
+    Dims d;
+    int st = check_shape(shape, &d);
+    if (st != NABLA_OK) return st;
+    if (params == nullptr) return NABLA_ERR_NULL;
+    const bool thr = params->mode == NABLA_DR_THRESHOLD;
+    if (!thr && params->mode != NABLA_DR_STATIC_RATIO) return NABLA_ERR_PARAM;
+    // the window, scale and flag rules of nabla_params (p is not used)
+    const nabla_params common{1.0f, params->sta_t, params->sta_h, params->sta_w, params->scale,
+                              params->flags};
+    if ((st = check_params(&common, true)) != NABLA_OK) return st;
+    if (params->flags & NABLA_DEBUG_TIMEOUT) return NABLA_ERR_PARAM;
+    if (!thr && (params->flags & NABLA_DEBUG_SCORES)) return NABLA_ERR_PARAM;  // no scores
+    if (!(params->gamma > 0.0 && params->gamma <= 1.0)) return NABLA_ERR_PARAM;
+    if (!(params->lambda >= 0.0 && params->lambda <= 1.0)) return NABLA_ERR_PARAM;
+    if (!(params->tau >= 0.0f)) return NABLA_ERR_PARAM;  // also rejects NaN; infinity keeps all
+    if ((st = check_mask_ptrs(&common, mask)) != NABLA_OK) return st;
+    if (thr) {
+        if (q == nullptr || k == nullptr) return NABLA_ERR_NULL;
+        if (!aligned16(q) || !aligned16(k)) return NABLA_ERR_ALIGN;
+    }
+    const int op = thr ? NABLA_OP_BUILD_MASK : NABLA_OP_ATTN_FWD;  // the latter: status only
+    if ((st = check_ws(d, op, workspace, workspace_bytes)) != NABLA_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
+    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
+    float *qbar = thr ? reinterpret_cast<float *>(w) : nullptr;
+    float *kbar_t = thr ? reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes) : nullptr;
+    const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
+    return cuda_status(nabla_launch_build_mask_dr(
+        d.BH, d.nb, d.D, shape->T, d.Hp, d.Wp, params->mode, params->gamma, params->lambda,
+        params->tau, params->scale, params->sta_t, params->sta_h, params->sta_w, params->flags, q,
+        k, qbar, kbar_t, mask->bits, mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
+        cols ? mask->col_cnt : nullptr, debug_scores(&common, mask), s));
 }
 
 int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,

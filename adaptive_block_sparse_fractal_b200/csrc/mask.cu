@@ -204,7 +204,51 @@ struct CutParams {
     int nb, T, Hp, Wp, wt, wh, ww;
     unsigned flags;
     float p, scale;
+    int mode;   // 0: CDF cut at p (NABLA); 1: logit threshold tau (DynamicRad)
+    float tau;  // mode 1: keep s_ij with max_j s_ij - s_ij <= tau (float32)
 };
+
+// Completes one bit row held in a warp's shared words sw[0 .. words) (the
+// selected blocks already set): ORs in the diagonal and the STA window
+// (section 手法: NABLA, "STA とのハイブリッド統合": |dt| <= wt/2, |dh| <= wh/2,
+// |dw| <= ww/2 in block coordinates, truncated at the grid border; enumerated
+// block by block over the clipped window), then writes the bit row, the
+// ascending row list and its count.  Called by all 32 lanes of the warp.
+__device__ __forceinline__ void finish_row(const CutParams &prm, int64_t bh, int i, uint32_t *sw,
+                                           uint32_t *__restrict__ bits,
+                                           uint16_t *__restrict__ row_idx,
+                                           int32_t *__restrict__ row_cnt) {
+    const int lane = threadIdx.x & 31, nb = prm.nb, words = (nb + 31) >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    __syncwarp();
+    if (lane == 0) atomicOr(sw + (i >> 5), 1u << (i & 31));
+    if (!(prm.flags & 1u)) {
+        const int HWp = prm.Hp * prm.Wp;
+        const int ti = i / HWp, hi = (i / prm.Wp) % prm.Hp, wi = i % prm.Wp;
+        const int t0 = max(0, ti - prm.wt / 2), t1 = min(prm.T - 1, ti + prm.wt / 2);
+        const int h0 = max(0, hi - prm.wh / 2), h1 = min(prm.Hp - 1, hi + prm.wh / 2);
+        const int w0 = max(0, wi - prm.ww / 2), w1 = min(prm.Wp - 1, wi + prm.ww / 2);
+        const int nh = h1 - h0 + 1, nw = w1 - w0 + 1;
+        const int cells = (t1 - t0 + 1) * nh * nw;
+        for (int c = lane; c < cells; c += 32) {
+            const int t = t0 + c / (nh * nw), h = h0 + (c / nw) % nh, w = w0 + c % nw;
+            const int j = (t * prm.Hp + h) * prm.Wp + w;
+            atomicOr(sw + (j >> 5), 1u << (j & 31));
+        }
+    }
+    __syncwarp();
+    uint32_t *brow = bits + (bh * nb + i) * words;
+    for (int w = lane; w < words; w += 32) brow[w] = sw[w];
+    uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
+    int cnt = 0;
+    for (int w = 0; w < words; ++w) {
+        const uint32_t word = sw[w];
+        if ((word >> lane) & 1u) lst[cnt + __popc(word & lt)] = static_cast<uint16_t>(w * 32 + lane);
+        cnt += __popc(word);
+    }
+    if (lane == 0) row_cnt[bh * nb + i] = cnt;
+    __syncwarp();  // sw is reused by the warp's next row
+}
 
 __device__ __forceinline__ uint32_t order_key(float s) {
     uint32_t b = __float_as_uint(s);
@@ -366,7 +410,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint32_t *hist = sH + warp * kHistWords;  // hi[256] | lo[256]
     uint32_t *sw = sW + warp * kMaxWords;
     int *ent = sE + warp * kCand;
-    const int HWp = prm.Hp * prm.Wp;
     for (int r = warp; r < rows_here; r += kWarps) {
         const int i = i0 + r;
         const float *srow = sS + r * nbp;
@@ -396,6 +439,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int o = 16; o > 0; o >>= 1) {
             smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
             smin = fminf(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+        }
+        if (prm.mode == 1) {
+            // logit threshold: keep the blocks within tau of the row's best
+            for (int e = 0; e < words; ++e) {
+                const float s = score(e * 32 + lane);
+                const unsigned keep = __ballot_sync(0xffffffffu, s > -INFINITY &&
+                                                                     __fsub_rn(smax, s) <= prm.tau);
+                if (lane == 0) sw[e] = keep;
+            }
+            finish_row(prm, bh, i, sw, bits, row_idx, row_cnt);
+            continue;
         }
         // bins over [0, span) of s_max - s; beyond 28 the masses are 0
         // (e^-28 * 2^40 < 1), so those blocks may share the last bin
@@ -591,34 +645,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         __syncwarp();
 
-        // the diagonal and the STA window
-        if (lane == 0) atomicOr(sw + (i >> 5), 1u << (i & 31));
-        if (!(prm.flags & 1u)) {
-            // the window clipped to the grid, enumerated block by block
-            const int ti = i / HWp, hi = (i / prm.Wp) % prm.Hp, wi = i % prm.Wp;
-            const int t0 = max(0, ti - prm.wt / 2), t1 = min(prm.T - 1, ti + prm.wt / 2);
-            const int h0 = max(0, hi - prm.wh / 2), h1 = min(prm.Hp - 1, hi + prm.wh / 2);
-            const int w0 = max(0, wi - prm.ww / 2), w1 = min(prm.Wp - 1, wi + prm.ww / 2);
-            const int nh = h1 - h0 + 1, nw = w1 - w0 + 1;
-            const int cells = (t1 - t0 + 1) * nh * nw;
-            for (int c = lane; c < cells; c += 32) {
-                const int t = t0 + c / (nh * nw), h = h0 + (c / nw) % nh, w = w0 + c % nw;
-                const int j = (t * prm.Hp + h) * prm.Wp + w;
-                atomicOr(sw + (j >> 5), 1u << (j & 31));
-            }
-        }
-        __syncwarp();
-        uint32_t *brow = bits + (bh * nb + i) * words;
-        for (int w = lane; w < words; w += 32) brow[w] = sw[w];
-        uint16_t *lst = row_idx + (bh * nb + i) * static_cast<int64_t>(nb);
-        int cnt = 0;
-        for (int w = 0; w < words; ++w) {
-            const uint32_t word = sw[w];
-            if ((word >> lane) & 1u) lst[cnt + __popc(word & lt)] = static_cast<uint16_t>(w * 32 + lane);
-            cnt += __popc(word);
-        }
-        if (lane == 0) row_cnt[bh * nb + i] = cnt;
-        __syncwarp();  // sw, the histogram and the list are reused by the next row
+        finish_row(prm, bh, i, sw, bits, row_idx, row_cnt);
     }
 }
 
@@ -646,6 +673,68 @@ __device__ __forceinline__ bool in_window(const BlockCoord &a, const BlockCoord 
                                           const CutParams &prm) {
     return abs(a.t - b.t) <= prm.wt / 2 && abs(a.h - b.h) <= prm.wh / 2 &&
            abs(a.w - b.w) <= prm.ww / 2;
+}
+
+// ---------------------------------------------------------------------------
+// DynamicRad static-ratio mask ("DynamicRad: Content-Adaptive Sparse Attention
+// for Long Video Diffusion", section 2.A, Static-Ratio mode): content-free.
+// Query block i = (t_i, q) keeps, in every frame t, the k(|t - t_i|) patches
+// nearest to its patch q (squared distance in patch units, then block index).
+// One CTA per (bh, patch position q): the patch ranks around q and the counts
+// k(dt) are computed once into shared memory, then one warp per frame t_i
+// builds the row of block (t_i, q).
+// ---------------------------------------------------------------------------
+struct RatioParams {
+    double gamma, lambda;
+};
+
+__global__ void __launch_bounds__(256) ratio_kernel(CutParams prm, RatioParams rp,
+                                                    uint32_t *__restrict__ bits,
+                                                    uint16_t *__restrict__ row_idx,
+                                                    int32_t *__restrict__ row_cnt) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int nb = prm.nb, T = prm.T, Wp = prm.Wp, HW = prm.Hp * prm.Wp;
+    const int words = (nb + 31) >> 5;
+    uint32_t *sW = reinterpret_cast<uint32_t *>(smem);            // [8][kMaxWords]
+    int *rank = reinterpret_cast<int *>(sW + 8 * kMaxWords);        // [HW]
+    int *kcnt = rank + HW;                                          // [T]
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t bh = blockIdx.x / HW;
+    const int q = static_cast<int>(blockIdx.x % HW);
+    const int qh = q / Wp, qw = q % Wp;
+    // (with one frame every row keeps its whole frame: no ranks needed)
+    for (int p = tid; T > 1 && p < HW; p += blockDim.x) {
+        const int dh = p / Wp - qh, dw = p % Wp - qw, dp = dh * dh + dw * dw;
+        int r = 0;
+        for (int p2 = 0; p2 < HW; ++p2) {
+            const int eh = p2 / Wp - qh, ew = p2 % Wp - qw, d2 = eh * eh + ew * ew;
+            r += (d2 < dp || (d2 == dp && p2 < p)) ? 1 : 0;
+        }
+        rank[p] = r;
+    }
+    for (int dt = tid; dt < T; dt += blockDim.x) {
+        double g = 1.0;
+        for (int n = 0; n < dt; ++n) g = __dmul_rn(g, rp.gamma);  // gamma^dt, dt factors
+        const double r = fmin(1.0, fmax(rp.lambda, g));
+        kcnt[dt] = static_cast<int>(fmin(ceil(__dmul_rn(r, static_cast<double>(HW))),
+                                         static_cast<double>(HW)));
+    }
+    __syncthreads();
+    uint32_t *sw = sW + warp * kMaxWords;
+    for (int ti = warp; ti < T; ti += 8) {
+        const int i = ti * HW + q;
+        for (int e = 0; e < words; ++e) {
+            const int j = e * 32 + lane;
+            bool keep = false;
+            if (j < nb) {
+                const int tj = j / HW, dt = tj > ti ? tj - ti : ti - tj;
+                keep = kcnt[dt] >= HW || rank[j - tj * HW] < kcnt[dt];
+            }
+            const unsigned b = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0) sw[e] = b;
+        }
+        finish_row(prm, bh, i, sw, bits, row_idx, row_cnt);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -781,7 +870,7 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, in
                                     uint16_t *col_idx, int32_t *col_cnt, float *scores,
                                     cudaStream_t stream, const void *q_grid, const void *k_grid) {
     using namespace nabla;
-    CutParams prm{nb, T, Hp, Wp, wt, wh, ww, flags, p, scale};
+    CutParams prm{nb, T, Hp, Wp, wt, wh, ww, flags, p, scale, 0, 0.f};
     cudaError_t err;
     const bool from_grid = q_grid != nullptr;
     const int bpc = 256 / (D / 8);
@@ -836,6 +925,60 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, in
                                            scores, stream)
                    : launch_score_cut<64>(grid, smem, qbar, kbar_t, prm, bits, row_idx, row_cnt,
                                           scores, stream);
+    if (err != cudaSuccess) return err;
+    if (col_idx) {
+        col_lists_kernel<<<col_grid, kColWarps * 32, 0, stream>>>(bits, col_idx, col_cnt, nb);
+        err = cudaGetLastError();
+    }
+    return err;
+}
+
+// DynamicRad-style masks (mode 0: static ratio, mode 1: logit threshold) in
+// the same list format; the threshold mode pools and scores like the NABLA
+// path.
+cudaError_t nabla_launch_build_mask_dr(int64_t BH, int nb, int D, int T, int Hp, int Wp, int mode,
+                                       double gamma, double lambda, float tau, float scale, int wt,
+                                       int wh, int ww, unsigned flags, const void *q,
+                                       const void *k, float *qbar, float *kbar_t, uint32_t *bits,
+                                       uint16_t *row_idx, int32_t *row_cnt, uint16_t *col_idx,
+                                       int32_t *col_cnt, float *scores, cudaStream_t stream) {
+    using namespace nabla;
+    CutParams prm{nb, T, Hp, Wp, wt, wh, ww, flags, 1.0f, scale, mode, tau};
+    cudaError_t err;
+    const int words = (nb + 31) / 32;
+    const dim3 col_grid(static_cast<unsigned>(BH * words));
+    if (flags & 2u) {  // the full window: every block
+        const int64_t rows = BH * nb;
+        sta_emit_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
+            prm, rows, bits, row_idx, row_cnt);
+    } else if (mode == 0) {
+        const int HW = Hp * Wp;
+        const size_t smem = sizeof(uint32_t) * 8 * kMaxWords + sizeof(int) * (HW + T);
+        ratio_kernel<<<static_cast<unsigned>(BH * HW), 256, smem, stream>>>(
+            prm, RatioParams{gamma, lambda}, bits, row_idx, row_cnt);
+    } else {
+        const int bpc = 256 / (D / 8);
+        const int64_t tiles = (nb + bpc - 1) / bpc;
+        const dim3 pool_grid(static_cast<unsigned>(2 * BH * tiles));
+        if (D == 128)
+            pool_kernel<128><<<pool_grid, 256, 0, stream>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
+                kbar_t, BH, nb);
+        else
+            pool_kernel<64><<<pool_grid, 256, 0, stream>>>(
+                static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar,
+                kbar_t, BH, nb);
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+        const size_t smem = nabla_score_cut_smem(nb, D);
+        const dim3 grid(static_cast<unsigned>(BH * ((nb + kRows - 1) / kRows)));
+        err = D == 128 ? launch_score_cut<128>(grid, smem, qbar, kbar_t, prm, bits, row_idx,
+                                               row_cnt, scores, stream)
+                       : launch_score_cut<64>(grid, smem, qbar, kbar_t, prm, bits, row_idx,
+                                              row_cnt, scores, stream);
+        if (err != cudaSuccess) return err;
+    }
+    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (col_idx) {
         col_lists_kernel<<<col_grid, kColWarps * 32, 0, stream>>>(bits, col_idx, col_cnt, nb);

@@ -21,8 +21,9 @@ MASK_BITS, MASK_ROW_IDX, MASK_ROW_CNT, MASK_COL_IDX, MASK_COL_CNT, MASK_SCORES =
 
 # every symbol include/nabla.h declares
 SYMBOLS = ("nabla_flatten", "nabla_workspace_size", "nabla_mask_bytes", "nabla_build_mask",
-           "nabla_build_mask_grid", "nabla_build_mask_static", "nabla_attn_fwd", "nabla_attn_bwd",
-           "nabla_status", "nabla_strerror")
+           "nabla_build_mask_grid", "nabla_build_mask_static", "nabla_build_mask_dr",
+           "nabla_attn_fwd", "nabla_attn_bwd", "nabla_status", "nabla_strerror")
+DR_STATIC_RATIO, DR_THRESHOLD = 0, 1
 
 
 class NablaError(RuntimeError):
@@ -37,6 +38,12 @@ class Shape(ctypes.Structure):
 
 class Params(ctypes.Structure):
     _fields_ = [("p", ctypes.c_float), ("sta_t", ctypes.c_int), ("sta_h", ctypes.c_int),
+                ("sta_w", ctypes.c_int), ("scale", ctypes.c_float), ("flags", ctypes.c_uint)]
+
+
+class DrParams(ctypes.Structure):
+    _fields_ = [("mode", ctypes.c_int), ("gamma", ctypes.c_double), ("lambda_", ctypes.c_double),
+                ("tau", ctypes.c_float), ("sta_t", ctypes.c_int), ("sta_h", ctypes.c_int),
                 ("sta_w", ctypes.c_int), ("scale", ctypes.c_float), ("flags", ctypes.c_uint)]
 
 
@@ -69,6 +76,8 @@ def lib():
         L.nabla_build_mask_grid.restype = I
         L.nabla_build_mask_static.argtypes = [P, P, P, P, P, P]
         L.nabla_build_mask_static.restype = I
+        L.nabla_build_mask_dr.argtypes = [P, P, P, P, P, P, SZ, P]
+        L.nabla_build_mask_dr.restype = I
         L.nabla_attn_fwd.argtypes = [P, P, P, P, P, P, P, P, P, SZ, P]
         L.nabla_attn_fwd.restype = I
         L.nabla_attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, P, P, SZ, P]
@@ -112,6 +121,14 @@ def params_of(p, window=(3, 3, 3), scale=None, D=None, flags=0):
         scale = D ** -0.5
     return Params(float(p), int(window[0]), int(window[1]), int(window[2]), float(scale),
                   int(flags))
+
+
+def dr_params_of(mode, gamma=1.0, lam=0.0, tau=0.0, window=(3, 3, 3), scale=None, D=None,
+                 flags=0):
+    if scale is None:
+        scale = D ** -0.5
+    return DrParams(int(mode), float(gamma), float(lam), float(tau), int(window[0]),
+                    int(window[1]), int(window[2]), float(scale), int(flags))
 
 
 def workspace_size(shape, op):
@@ -178,6 +195,27 @@ def build_mask(shape, params, q, k, mask=None, ws=None):
     _check(lib().nabla_build_mask(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k),
                                   ctypes.byref(ms), _ptr(ws), ws.numel(), _stream(q)),
            "nabla_build_mask")
+    return mask
+
+
+def build_mask_dr(shape, params, q=None, k=None, mask=None, ws=None, device=None):
+    """DynamicRad-style mask (static ratio or logit threshold) in the same
+    format; q and k are needed by the threshold mode only."""
+    thr = params.mode == DR_THRESHOLD
+    if thr:
+        _need(q, torch.bfloat16, "q")
+        _need(k, torch.bfloat16, "k")
+        device = q.device
+    cols = bool(params.flags & EMIT_COLS)
+    dbg = bool(params.flags & DEBUG_SCORES)
+    mask = alloc_mask(shape, device, cols, dbg) if mask is None else mask
+    if ws is None:
+        ws = workspace(shape, OP_BUILD_MASK if thr else OP_ATTN_FWD, device)
+    ms = _mask_struct(mask)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(ws.device).cuda_stream)
+    _check(lib().nabla_build_mask_dr(ctypes.byref(shape), ctypes.byref(params), _ptr(q), _ptr(k),
+                                     ctypes.byref(ms), _ptr(ws), ws.numel(), stream),
+           "nabla_build_mask_dr")
     return mask
 
 

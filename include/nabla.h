@@ -215,6 +215,41 @@ int nabla_build_mask_static(const nabla_shape *shape, const nabla_params *params
                             const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
                             nabla_stream_t stream);
 
+/* DynamicRad-style masks in the same format ("DynamicRad: Content-Adaptive
+ * Sparse Attention for Long Video Diffusion", section 2.A "Dual-Mode
+ * Strategy"): a second pair of mask producers for the same attention calls.
+ * Per (batch, head) and query block i = (t_i, ph_i, pw_i):
+ *   NABLA_DR_STATIC_RATIO (content-free; q and k are not read, may be NULL):
+ *     in frame t_j, with dt = |t_j - t_i|, keep the
+ *       k(dt) = ceil(min(1, max(lambda, gamma^dt)) * Hp * Wp)
+ *     patches nearest to (ph_i, pw_i): ascending (ph - ph_i)^2 + (pw - pw_i)^2,
+ *     equal distances by ascending block index.  gamma^dt is a product of dt
+ *     factors in float64 and k a float64 product rounded up.
+ *   NABLA_DR_THRESHOLD (content-adaptive): with the pooled scores s_ij of
+ *     nabla_build_mask (same float32 arithmetic), keep j where the float32
+ *     difference max_j s_ij - s_ij <= tau: the blocks whose pre-softmax logit
+ *     is within tau of the row's best (softmax weight >= e^-tau of the best).
+ *   M_ij = selected OR STA window (unless NABLA_NO_STA) OR (i == j).
+ * gamma in (0, 1], lambda in [0, 1], tau >= 0 (infinity keeps everything);
+ * other fields and flags (NABLA_NO_STA, NABLA_EMIT_COLS, NABLA_DEBUG_SCORES in
+ * the threshold mode) as nabla_params.  Workspace: as nabla_build_mask for
+ * the threshold mode; the static mode needs only the status region
+ * (nabla_workspace_size(shape, NABLA_OP_ATTN_FWD) bytes suffice). */
+#define NABLA_DR_STATIC_RATIO 0
+#define NABLA_DR_THRESHOLD 1
+typedef struct {
+    int mode;
+    double gamma, lambda;
+    float tau;
+    int sta_t, sta_h, sta_w;
+    float scale;
+    unsigned flags;
+} nabla_dr_params;
+
+int nabla_build_mask_dr(const nabla_shape *shape, const nabla_dr_params *params,
+                        const nabla_bf16 *q, const nabla_bf16 *k, const nabla_mask *mask,
+                        void *workspace, size_t workspace_bytes, nabla_stream_t stream);
+
 /* Block-sparse attention forward over M (bullet "拡張": attention is
  * computed for the kept blocks only).  For query token n of block i:
  *   o_n   = sum over tokens m of blocks j in row i of M of

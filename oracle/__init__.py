@@ -61,6 +61,12 @@ def _declare(L):
     L.oracle_mask.restype = None
     L.oracle_mask.argtypes = [_P, _P, _I64, _I64, _I, _I, _I, _F, _F, _I, _I, _I, _U,
                               _P, _P, _P, _P, _P, _P, _P]
+    L.oracle_dr_static.restype = None
+    L.oracle_dr_static.argtypes = [_I64, _I64, _I, _I, _I, _D, _D, _I, _I, _I, _U,
+                                   _P, _P, _P, _P, _P, _P]
+    L.oracle_dr_threshold.restype = None
+    L.oracle_dr_threshold.argtypes = [_P, _P, _I64, _I64, _I, _I, _I, _F, _F, _I, _I, _I, _U,
+                                      _P, _P, _P, _P, _P, _P]
     L.oracle_cut_row_f64.restype = _I64
     L.oracle_cut_row_f64.argtypes = [_P, _I64, _D, _P]
     L.oracle_cut_row_fixed.restype = _I64
@@ -216,6 +222,33 @@ def mask_f64(qbar, kbar, grid, p, scale, window=(3, 3, 3), flags=0, cols=True):
                           *window, flags, _ptr(m["bits"]), _ptr(m["row_idx"]),
                           _ptr(m["row_cnt"]), _ptr(m.get("col_idx")), _ptr(m.get("col_cnt")),
                           _ptr(m["adapt_cnt"]), _ptr(m["cum_before"]), _ptr(m["cum_at"]))
+    return m
+
+
+def dr_static(BH, grid, gamma, lam, window=(3, 3, 3), flags=0, cols=True):
+    """DynamicRad static-ratio mask (content-free) for BH heads of a grid
+    (T, Hp, Wp) in blocks."""
+    T, Hp, Wp = grid
+    nb = T * Hp * Wp
+    m = _mask_buffers(BH, nb, cols)
+    lib().oracle_dr_static(BH, nb, T, Hp, Wp, float(gamma), float(lam), *window, flags,
+                           _ptr(m["bits"]), _ptr(m["row_idx"]), _ptr(m["row_cnt"]),
+                           _ptr(m.get("col_idx")), _ptr(m.get("col_cnt")), _ptr(m["adapt_cnt"]))
+    return m
+
+
+def dr_threshold(qbar, kbar, grid, tau, scale, window=(3, 3, 3), flags=0, cols=True):
+    """DynamicRad logit-threshold mask from float32 pooled means."""
+    qbar = _c(qbar, np.float32)
+    kbar = _c(kbar, np.float32)
+    BH, nb, D = qbar.shape
+    T, Hp, Wp = grid
+    assert T * Hp * Wp == nb
+    m = _mask_buffers(BH, nb, cols)
+    lib().oracle_dr_threshold(_ptr(qbar), _ptr(kbar), BH, nb, D, Hp, Wp, np.float32(tau),
+                              np.float32(scale), *window, flags, _ptr(m["bits"]),
+                              _ptr(m["row_idx"]), _ptr(m["row_cnt"]), _ptr(m.get("col_idx")),
+                              _ptr(m.get("col_cnt")), _ptr(m["adapt_cnt"]))
     return m
 
 

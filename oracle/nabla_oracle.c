@@ -415,6 +415,105 @@ void oracle_mask(const float *qbar, const float *kbar, int64_t BH, int64_t nb, i
     free(keep_all);
 }
 
+/* ------------------------------------------------------------------------ */
+/* DynamicRad-style masks ("DynamicRad: Content-Adaptive Sparse Attention     */
+/* for Long Video Diffusion", section 2.A "Dual-Mode Strategy"), emitted in   */
+/* the same format: selected OR STA OR diagonal.                              */
+/* ------------------------------------------------------------------------ */
+
+typedef struct {
+    int64_t d; /* squared distance to the query's patch, in patch units */
+    int64_t p; /* patch index in the frame; smaller first on equal d */
+} patch_item;
+
+static int patch_cmp(const void *a, const void *b)
+{
+    const patch_item *x = (const patch_item *)a, *y = (const patch_item *)b;
+    if (x->d != y->d) return x->d < y->d ? -1 : 1;
+    return (x->p < y->p) ? -1 : (x->p > y->p);
+}
+
+/* Static-Ratio mode (no content scoring; a fixed retention ratio by temporal
+ * distance).  Query block i = (t_i, ph_i, pw_i) keeps, in frame t with
+ * dt = |t - t_i|, the k(dt) = ceil(min(1, max(lambda, gamma^dt)) * Hp*Wp)
+ * patches nearest to (ph_i, pw_i) (squared distance, then patch index);
+ * gamma^dt is the product of dt factors gamma in double precision.
+ * adapt_cnt (may be NULL) gets the number of selected blocks per row. */
+void oracle_dr_static(int64_t BH, int64_t nb, int T, int Hp, int Wp, double gamma, double lambda,
+                      int wt, int wh, int ww, unsigned flags, uint32_t *bits, uint16_t *row_idx,
+                      int32_t *row_cnt, uint16_t *col_idx, int32_t *col_cnt, int32_t *adapt_cnt)
+{
+    int64_t HW = (int64_t)Hp * Wp;
+    uint8_t *keep_all = (uint8_t *)calloc((size_t)(BH * nb * nb), 1);
+#pragma omp parallel
+    {
+        patch_item *order = (patch_item *)malloc(sizeof(patch_item) * (size_t)HW);
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < nb; ++i) {
+                int64_t ti = i / HW, qh = (i % HW) / Wp, qw = i % Wp;
+                uint8_t *keep = keep_all + (bh * nb + i) * nb;
+                for (int64_t p = 0; p < HW; ++p) {
+                    int64_t dh = p / Wp - qh, dw = p % Wp - qw;
+                    order[p].d = dh * dh + dw * dw;
+                    order[p].p = p;
+                }
+                qsort(order, (size_t)HW, sizeof(patch_item), patch_cmp);
+                int32_t c = 0;
+                for (int64_t t = 0; t < T; ++t) {
+                    int64_t dt = t > ti ? t - ti : ti - t;
+                    double g = 1.0;
+                    for (int64_t n = 0; n < dt; ++n) g = g * gamma;
+                    double r = fmin(1.0, fmax(lambda, g));
+                    int64_t k = (int64_t)fmin(ceil(r * (double)HW), (double)HW);
+                    for (int64_t m = 0; m < k; ++m) keep[t * HW + order[m].p] = 1;
+                    c += (int32_t)k;
+                }
+                if (adapt_cnt) adapt_cnt[bh * nb + i] = c;
+            }
+        free(order);
+    }
+    emit_mask(keep_all, BH, nb, Hp, Wp, wt, wh, ww, flags, bits, row_idx, row_cnt, col_idx,
+              col_cnt);
+    free(keep_all);
+}
+
+/* Dynamic-Threshold mode (pre-softmax logits as the importance proxy): with
+ * the decision-precision pooled scores s_ij (scores_row_f32), keep j where the
+ * float32 difference max_j s_ij - s_ij is at most tau. */
+void oracle_dr_threshold(const float *qbar, const float *kbar, int64_t BH, int64_t nb, int D,
+                         int Hp, int Wp, float tau, float scale, int wt, int wh, int ww,
+                         unsigned flags, uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
+                         uint16_t *col_idx, int32_t *col_cnt, int32_t *adapt_cnt)
+{
+    uint8_t *keep_all = (uint8_t *)calloc((size_t)(BH * nb * nb), 1);
+#pragma omp parallel
+    {
+        float *score = (float *)malloc(sizeof(float) * (size_t)nb);
+#pragma omp for collapse(2) schedule(dynamic, 16)
+        for (int64_t bh = 0; bh < BH; ++bh)
+            for (int64_t i = 0; i < nb; ++i) {
+                scores_row_f32(qbar + (bh * nb + i) * D, kbar + bh * nb * D, nb, D, scale, score);
+                float smax = -INFINITY;
+                for (int64_t j = 0; j < nb; ++j) smax = fmaxf(smax, score[j]);
+                uint8_t *keep = keep_all + (bh * nb + i) * nb;
+                int32_t c = 0;
+                for (int64_t j = 0; j < nb; ++j) {
+                    float gap = smax - score[j];
+                    if (gap <= tau) {
+                        keep[j] = 1;
+                        ++c;
+                    }
+                }
+                if (adapt_cnt) adapt_cnt[bh * nb + i] = c;
+            }
+        free(score);
+    }
+    emit_mask(keep_all, BH, nb, Hp, Wp, wt, wh, ww, flags, bits, row_idx, row_cnt, col_idx,
+              col_cnt);
+    free(keep_all);
+}
+
 /* Stand-alone cuts on given score rows (used by the brute-force pins). */
 int64_t oracle_cut_row_f64(const double *score, int64_t nb, double p, uint8_t *keep)
 {

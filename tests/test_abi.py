@@ -120,6 +120,44 @@ def test_build_mask_grid_rejects_on_host(L):
     assert g(a, b, c, d, params=nabla.params_of(1.5, (3, 3, 3), D=128)) == nabla.ERR_PARAM
 
 
+def test_debug_scores_needs_its_buffer(L):
+    s = _shape()
+    assert nabla.mask_bytes(s, nabla.MASK_SCORES) == 40 * 1200 * 1200 * 4
+    dbg = nabla.params_of(0.7, (3, 3, 3), D=128, flags=nabla.DEBUG_SCORES)
+    assert _build(L, s, dbg) == nabla.ERR_NULL  # mask.scores is NULL
+    m = nabla.MaskStruct(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert _build(L, s, dbg, mask=m, ws_bytes=1024) == nabla.ERR_WORKSPACE  # got past the NULL check
+
+
+def _dr(L, params, shape=None, q=FAKE, k=FAKE, mask=None, ws=FAKE, ws_bytes=1 << 40):
+    m = _mask() if mask is None else mask
+    s = _shape() if shape is None else shape
+    return L.nabla_build_mask_dr(ctypes.byref(s), ctypes.byref(params), q, k, ctypes.byref(m), ws,
+                                 ws_bytes, None)
+
+
+def test_dynamicrad_masks_reject_on_host(L):
+    ratio = lambda **kw: nabla.dr_params_of(nabla.DR_STATIC_RATIO, D=128, **kw)
+    thr = lambda **kw: nabla.dr_params_of(nabla.DR_THRESHOLD, D=128, **kw)
+    for bad in (ratio(gamma=0.0), ratio(gamma=1.5), ratio(gamma=0.5, lam=-0.1),
+                ratio(gamma=0.5, lam=1.1), thr(tau=-1.0), thr(tau=float("nan")),
+                ratio(gamma=0.5, window=(2, 3, 3)),
+                ratio(gamma=0.5, flags=nabla.DEBUG_SCORES),  # the static mode has no scores
+                thr(tau=1.0, flags=nabla.DEBUG_TIMEOUT)):
+        assert _dr(L, bad) == nabla.ERR_PARAM
+    bad_mode = thr(tau=1.0)
+    bad_mode.mode = 7
+    assert _dr(L, bad_mode) == nabla.ERR_PARAM
+    assert _dr(L, thr(tau=1.0), q=None) == nabla.ERR_NULL         # the threshold mode reads q, k
+    assert _dr(L, thr(tau=1.0), k=FAKE_ODD) == nabla.ERR_ALIGN
+    assert _dr(L, thr(tau=1.0), ws_bytes=1024) == nabla.ERR_WORKSPACE
+    # the static mode reads neither q nor k and needs only the status region
+    assert _dr(L, ratio(gamma=0.5), q=None, k=None, ws_bytes=16) == nabla.ERR_WORKSPACE
+    assert _dr(L, ratio(gamma=0.5), shape=_shape(P=4)) == nabla.ERR_SHAPE
+    assert L.nabla_build_mask_dr(ctypes.byref(_shape()), None, FAKE, FAKE, ctypes.byref(_mask()),
+                                 FAKE, 1 << 40, None) == nabla.ERR_NULL
+
+
 def test_attention_rejects_on_host(L):
     s, good = _shape(), nabla.params_of(0.7, (3, 3, 3), D=128)
     m = _mask()
@@ -145,6 +183,9 @@ def test_flatten_rejects_on_host(L):
     assert f(FAKE, ctypes.c_void_p(0x20000), 1, 2, 16, 16, 8, 24, 0, None) == nabla.ERR_ALIGN
     assert f(FAKE, ctypes.c_void_p(0x20000), 1, 2, 16, 12, 8, 256, 0, None) == nabla.ERR_SHAPE
     assert f(FAKE, FAKE, 1, 2, 16, 16, 8, 256, 0, None) == nabla.ERR_PARAM  # in place
+    # partially overlapping buffers (out starts inside in)
+    assert f(FAKE, ctypes.c_void_p(0x10000 + 4096), 1, 2, 16, 16, 8, 256, 0, None) == \
+        nabla.ERR_PARAM
     # empty inputs are a successful no-op
     assert f(FAKE, ctypes.c_void_p(0x20000), 0, 2, 16, 16, 8, 256, 0, None) == nabla.OK
 
