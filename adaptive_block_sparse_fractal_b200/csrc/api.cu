@@ -23,27 +23,17 @@ cudaError_t nabla_launch_build_mask_dr(int64_t BH, int nb, int D, int T, int Hp,
                                        const void *k, float *qbar, float *kbar_t, uint32_t *bits,
                                        uint16_t *row_idx, int32_t *row_cnt, uint16_t *col_idx,
                                        int32_t *col_cnt, float *scores, cudaStream_t stream);
-cudaError_t nabla_launch_attn_fwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
-                                      const void *k, const void *v, const uint16_t *row_idx,
-                                      const int32_t *row_cnt, void *o, float *lse,
-                                      cudaStream_t stream);
-cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
-                                        const void *q, const void *k, const void *v,
+cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int D, int Hp, int Wp, int T,
+                                        float scale, const void *q, const void *k, const void *v,
                                         const uint32_t *bits, void *o, float *lse, int *status,
                                         int force_timeout, cudaStream_t stream);
-cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
-                                        const void *q, const void *k, const void *v,
+cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int D, int Hp, int Wp, int T,
+                                        float scale, const void *q, const void *k, const void *v,
                                         const void *o, const void *dout, const float *lse,
                                         const uint16_t *row_idx, const int32_t *row_cnt,
                                         const uint16_t *col_idx, const int32_t *col_cnt,
                                         void *dq, void *dk, void *dv, float *dl, float *l2,
                                         int *status, int force_timeout, cudaStream_t stream);
-cudaError_t nabla_launch_attn_bwd_mma(int64_t BH, int nb, int D, float scale, const void *q,
-                                      const void *k, const void *v, const void *o,
-                                      const void *dout, const float *lse, const uint16_t *row_idx,
-                                      const int32_t *row_cnt, const uint16_t *col_idx,
-                                      const int32_t *col_cnt, void *dq, void *dk, void *dv,
-                                      float *dl, cudaStream_t stream);
 
 namespace {
 
@@ -304,14 +294,9 @@ int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const n
     if ((st = check_ws(d, NABLA_OP_ATTN_FWD, workspace, workspace_bytes)) != NABLA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
-    if (d.D == 128) {
-        const int T = shape->T;
-        return cuda_status(nabla_launch_attn_fwd_sm100(
-            d.BH, d.nb, d.Hp, d.Wp, T, params->scale, q, k, v, mask->bits, o, lse,
-            static_cast<int *>(workspace), (params->flags & NABLA_DEBUG_TIMEOUT) ? 1 : 0, s));
-    }
-    return cuda_status(nabla_launch_attn_fwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v,
-                                                 mask->row_idx, mask->row_cnt, o, lse, s));
+    return cuda_status(nabla_launch_attn_fwd_sm100(
+        d.BH, d.nb, d.D, d.Hp, d.Wp, shape->T, params->scale, q, k, v, mask->bits, o, lse,
+        static_cast<int *>(workspace), (params->flags & NABLA_DEBUG_TIMEOUT) ? 1 : 0, s));
 }
 
 int nabla_attn_bwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,
@@ -337,17 +322,12 @@ int nabla_attn_bwd(const nabla_shape *shape, const nabla_params *params, const n
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
     float *dl = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + kStatusBytes);
-    if (d.D == 128) {
-        float *l2 = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(dl) +
-                                              round256(sizeof(float) * d.BH * d.N));
-        return cuda_status(nabla_launch_attn_bwd_sm100(
-            d.BH, d.nb, d.Hp, d.Wp, shape->T, params->scale, q, k, v, o, dout, lse, mask->row_idx,
-            mask->row_cnt, mask->col_idx, mask->col_cnt, dq, dk, dv, dl, l2,
-            static_cast<int *>(workspace), (params->flags & NABLA_DEBUG_TIMEOUT) ? 1 : 0, s));
-    }
-    return cuda_status(nabla_launch_attn_bwd_mma(d.BH, d.nb, d.D, params->scale, q, k, v, o,
-                                                 dout, lse, mask->row_idx, mask->row_cnt,
-                                                 mask->col_idx, mask->col_cnt, dq, dk, dv, dl, s));
+    float *l2 = reinterpret_cast<float *>(reinterpret_cast<unsigned char *>(dl) +
+                                          round256(sizeof(float) * d.BH * d.N));
+    return cuda_status(nabla_launch_attn_bwd_sm100(
+        d.BH, d.nb, d.D, d.Hp, d.Wp, shape->T, params->scale, q, k, v, o, dout, lse,
+        mask->row_idx, mask->row_cnt, mask->col_idx, mask->col_cnt, dq, dk, dv, dl, l2,
+        static_cast<int *>(workspace), (params->flags & NABLA_DEBUG_TIMEOUT) ? 1 : 0, s));
 }
 
 int nabla_status(const void *workspace, nabla_stream_t stream) {

@@ -1,4 +1,6 @@
-// Block-sparse attention backward on tcgen05 tensor cores, head dim 128.
+// Block-sparse attention backward on tcgen05 tensor cores, head dim D = 128 or
+// 64 (one template; shared-memory tiles hold each 64-feature half of D as one
+// 128-byte swizzle atom column).
 //
 // "NABLA: Neighborhood Adaptive Block-Level Attention": training runs through
 // the same block-sparse attention (section 主な貢献, "二段階の加速"), so its
@@ -28,25 +30,25 @@ namespace bwd100 {
 
 using namespace sm100;
 
-constexpr int kD = 128;
 constexpr int kMaxNbBwd = 2048;
-constexpr uint32_t kHalfTile = 16384;  // 64 rows x 128 features bf16
-constexpr uint32_t kPairTile = 32768;  // 128 rows x 128 features bf16
+constexpr uint32_t kHalfTile = 16384;  // 128 rows x 64 features bf16 (one half of D)
 
 // ---------------------------------------------------------------------------
-// preprocess: D_n = dO_n . O_n and lse_n * log2(e), 16 threads per row
+// preprocess: D_n = dO_n . O_n and lse_n * log2(e), D/8 threads per row
 // ---------------------------------------------------------------------------
+template <int D>
 __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restrict__ o,
                                                   const __nv_bfloat16 *__restrict__ dout,
                                                   const float *__restrict__ lse,
                                                   float *__restrict__ dl, float *__restrict__ l2,
                                                   int64_t rows) {
-    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 4;
-    const int sub = threadIdx.x & 15;
+    constexpr int TPR = D / 8;  // threads per row, 8 features each
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPR;
+    const int sub = threadIdx.x % TPR;
     float acc = 0.f;
     if (row < rows) {
-        const int4 a = *reinterpret_cast<const int4 *>(o + row * kD + sub * 8);
-        const int4 b = *reinterpret_cast<const int4 *>(dout + row * kD + sub * 8);
+        const int4 a = *reinterpret_cast<const int4 *>(o + row * D + sub * 8);
+        const int4 b = *reinterpret_cast<const int4 *>(dout + row * D + sub * 8);
         const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
         const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&b);
 #pragma unroll
@@ -57,7 +59,7 @@ __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restric
         }
     }
 #pragma unroll
-    for (int off = 1; off < 16; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    for (int off = 1; off < TPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (row < rows && sub == 0) {
         // stored negated, the form the packed exponent and difference take
         dl[row] = -acc;
@@ -70,21 +72,29 @@ __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restric
 // ---------------------------------------------------------------------------
 constexpr int kStages = 3;
 constexpr int kKvThreads = 320;
-constexpr uint32_t kStageBytes = 33792;  // Q 16 KB + dO 16 KB + L2 256 B + D 256 B (+ pad)
-constexpr uint32_t KV_K = 0, KV_V = 32768;
-constexpr uint32_t KV_RING = 65536;
-constexpr uint32_t KV_U = KV_RING + kStages * kStageBytes;  // union list
-constexpr uint32_t KV_UF = KV_U + 2 * (kMaxNbBwd + 8);
-constexpr uint32_t KV_CB = ((KV_UF + kMaxNbBwd + 8 + 15) / 16) * 16;  // column bits [2][64]
-constexpr uint32_t KV_BAR = KV_CB + 2 * 256;
-constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
-constexpr uint32_t KV_INT = KV_BAR + 8 * kKvBars;
-constexpr uint32_t kKvSmem = KV_INT + 16 + 1024;
+// shared memory of the dK/dV kernel for head dim D: K and V of the key pair
+// (resident), then a ring of query stages (Q, dO, -L log2 e, -D)
+template <int D>
+struct KvLayout {
+    static constexpr int kHalves = D / 64;
+    static constexpr uint32_t kQBytes = 64u * D * 2;                   // one query block
+    static constexpr uint32_t kStageBytes = ((2 * kQBytes + 512 + 1023) / 1024) * 1024;
+    static constexpr uint32_t KV_K = 0, KV_V = kHalves * kHalfTile;
+    static constexpr uint32_t KV_RING = 2 * kHalves * kHalfTile;
+    static constexpr uint32_t KV_U = KV_RING + kStages * kStageBytes;  // union list
+    static constexpr uint32_t KV_UF = KV_U + 2 * (kMaxNbBwd + 8);
+    static constexpr uint32_t KV_CB = ((KV_UF + kMaxNbBwd + 8 + 15) / 16) * 16;  // col bits [2][64]
+    static constexpr uint32_t KV_BAR = KV_CB + 2 * 256;
+    static constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+    static constexpr uint32_t KV_INT = KV_BAR + 8 * kKvBars;
+    static constexpr uint32_t kKvSmem = KV_INT + 16 + 1024;
+};
 
 // TMEM columns: S^T(t) [64 (t&1), +64), dP^T(t) [128 + 64 (t&1), +64),
-// dV [256, 384), dK [384, 512).  Warpgroup qg handles queries [32 qg, +32) of
-// the tile and writes bf16 P^T and dS^T for them over the first 16 of its
-// own S^T and dP^T columns, where the dV and dK MMAs read them.
+// dV [256, 256 + D), dK [384, 384 + D).  Warpgroup qg handles queries
+// [32 qg, +32) of the tile and writes bf16 P^T and dS^T for them over the
+// first 16 of its own S^T and dP^T columns, where the dV and dK MMAs read them.
+template <int D>
 __global__ void __launch_bounds__(kKvThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -93,6 +103,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 __nv_bfloat16 *__restrict__ dk, __nv_bfloat16 *__restrict__ dv,
                 int *__restrict__ status, int nb, int Hp, int Wp, int T, float c, float scale,
                 uint32_t wait_limit, int force_timeout) {
+    using L = KvLayout<D>;
+    constexpr int kHalves = L::kHalves;
+    constexpr uint32_t kQBytes = L::kQBytes, kStageBytes = L::kStageBytes;
+    constexpr uint32_t KV_K = L::KV_K, KV_V = L::KV_V, KV_RING = L::KV_RING, KV_U = L::KV_U,
+                       KV_UF = L::KV_UF, KV_CB = L::KV_CB, KV_BAR = L::KV_BAR, KV_INT = L::KV_INT;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
@@ -170,8 +185,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         prefetch_tmap(&tv);
         prefetch_tmap(&tdo);
         const int ya = row_base + jA * kBlk, yb = row_base + (jB >= 0 ? jB : jA) * kBlk;
-        mbar_expect_tx(kv_full, 2 * kPairTile);
-        for (int dh = 0; dh < 2; ++dh) {
+        mbar_expect_tx(kv_full, 2 * kHalves * kHalfTile);
+        for (int dh = 0; dh < kHalves; ++dh) {
             tma_load_2d(sb + KV_K + dh * kHalfTile, &tk, kv_full, 64 * dh, ya);
             tma_load_2d(sb + KV_K + dh * kHalfTile + 8192, &tk, kv_full, 64 * dh, yb);
             tma_load_2d(sb + KV_V + dh * kHalfTile, &tv, kv_full, 64 * dh, ya);
@@ -184,13 +199,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const uint32_t dst = sb + KV_RING + s * kStageBytes;
             const int i = uList[t];
             const int y = row_base + i * kBlk;
-            mbar_expect_tx(&st_full[s], 2 * kHalfTile + 512);
-            tma_load_2d(dst, &tq, &st_full[s], 0, y);
-            tma_load_2d(dst + 8192, &tq, &st_full[s], 64, y);
-            tma_load_2d(dst + 16384, &tdo, &st_full[s], 0, y);
-            tma_load_2d(dst + 24576, &tdo, &st_full[s], 64, y);
-            bulk_load(dst + 32768, l2 + y, 256, &st_full[s]);
-            bulk_load(dst + 33024, dl + y, 256, &st_full[s]);
+            mbar_expect_tx(&st_full[s], 2 * kQBytes + 512);
+            for (int h = 0; h < kHalves; ++h) {  // [Q halves][dO halves], 8 KB each
+                tma_load_2d(dst + h * 8192, &tq, &st_full[s], 64 * h, y);
+                tma_load_2d(dst + kQBytes + h * 8192, &tdo, &st_full[s], 64 * h, y);
+            }
+            bulk_load(dst + 2 * kQBytes, l2 + y, 256, &st_full[s]);
+            bulk_load(dst + 2 * kQBytes + 256, dl + y, 256, &st_full[s]);
         }
         wait_plain(kv_full, 0, wait_limit);
         for (int u = t > kStages ? t - kStages : 0; u < t; ++u)
@@ -198,7 +213,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     } else if (warp == 1) {
         // MMA issuer: whole warp, one elected lane issues
         constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // K . Q^T, V . dO^T
-        constexpr uint32_t kIdG = idesc_bf16(128, 128, 0, 1);   // P^T . dO, dS^T . Q
+        constexpr uint32_t kIdG = idesc_bf16(128, D, 0, 1);     // P^T . dO, dS^T . Q
         auto SdP = [&](int t) -> bool {
             const int s = t % kStages;
             if (!warp_wait(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
@@ -206,13 +221,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
+            for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
                 const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
                 mma_ss_warp(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
                             desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
                 mma_ss_warp(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
-                            desc_sw128(st + 16384 + kb, 16, 1024), kIdS, kk > 0);
+                            desc_sw128(st + kQBytes + kb, 16, 1024), kIdS, kk > 0);
             }
             mma_commit_warp(&s_full[t & 1]);
             return true;
@@ -227,7 +242,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             for (int kk = 0; kk < 64 / 16; ++kk) {  // queries 16kk.. at column 32(kk/2) + 8(kk%2)
                 const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
                 const uint32_t col = (t & 1) * 64 + 32 * (kk >> 1) + 8 * (kk & 1);
-                mma_ts_warp(tmem + 256, tmem + col, desc_sw128(st + 16384 + kk * 2048, 8192, 1024),
+                mma_ts_warp(tmem + 256, tmem + col, desc_sw128(st + kQBytes + kk * 2048, 8192, 1024),
                             kIdG, acc);
                 mma_ts_warp(tmem + 384, tmem + 128 + col, desc_sw128(st + kk * 2048, 8192, 1024),
                             kIdG, acc);
@@ -261,7 +276,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             uint32_t pk[16], dk2[16];  // packed bf16 pairs of P^T and dS^T
             if (valid) {
                 const float4 *L4 = reinterpret_cast<const float4 *>(
-                    sm + KV_RING + (t % kStages) * kStageBytes + 32768 + 128 * qg);
+                    sm + KV_RING + (t % kStages) * kStageBytes + 2 * kQBytes + 128 * qg);
                 const float4 *D4 = L4 + 16;  // D follows L2 at +256 bytes
                 float sv[32], dp[32];
                 tmem_ld32(scol, sv);
@@ -307,10 +322,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             // warpgroup 0 writes the dV row, warpgroup 1 the dK row of key tw
             const int64_t row = bh * N + static_cast<int64_t>(jm) * kBlk + (tw & 63);
             const bool live = all_ok && ntiles > 0;
-            __nv_bfloat16 *dst = (qg ? dk : dv) + row * kD;
+            __nv_bfloat16 *dst = (qg ? dk : dv) + row * D;
             const float mul = qg ? scale : 1.f;
 #pragma unroll
-            for (int part = 0; part < 4; ++part) {
+            for (int part = 0; part < D / 32; ++part) {
                 float v[32];
                 if (live) {
                     tmem_ld32(tmem + lane_base + 256 + 128 * qg + 32 * part, v);
@@ -353,20 +368,26 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // writes their bf16 dS over its own S columns [32 g, 32 g + 16).
 // Queries of the pair whose own row does not keep a key block get dS = 0.
 // TMEM columns: buffer b in [128 b, 128 b + 128) holds S (64) then dP (64);
-// dQ [256, 384), Q [384, 448), dO [448, 512).
+// dQ [256, 256 + D), Q [384, 384 + D/2), dO [448, 448 + D/2).
 constexpr int kDqThreads = 320;
-constexpr int kDqRing = 6;
-constexpr uint32_t kDqSlot = 32768;  // K block 16 KB + V block 16 KB
 constexpr uint32_t kColDQ = 256, kColQ = 384, kColDO = 448;
-constexpr uint32_t DQ_RING = 0;
-constexpr uint32_t DQ_RB = DQ_RING + kDqRing * kDqSlot;   // row bits [2][64]
-constexpr uint32_t DQ_U = DQ_RB + 2 * 256;                // union list u16
-constexpr uint32_t DQ_UF = DQ_U + 2 * (kMaxNbBwd + 8);    // membership per entry
-constexpr uint32_t DQ_BAR = ((DQ_UF + kMaxNbBwd + 8 + 7) / 8) * 8;
-constexpr int kDqBars = 2 * kDqRing + 2 + 2 + 1 + 1 + 1;
-constexpr uint32_t DQ_INT = DQ_BAR + 8 * kDqBars;
-constexpr uint32_t kDqSmem = DQ_INT + 16 + 1024;
+template <int D>
+struct DqLayout {
+    static constexpr int kHalves = D / 64;
+    static constexpr int kDqRing = D == 128 ? 6 : 10;
+    static constexpr uint32_t kBlockBytes = 64u * D * 2;       // one K or V block
+    static constexpr uint32_t kDqSlot = 2 * kBlockBytes;       // K block + V block
+    static constexpr uint32_t DQ_RING = 0;
+    static constexpr uint32_t DQ_RB = DQ_RING + kDqRing * kDqSlot;   // row bits [2][64]
+    static constexpr uint32_t DQ_U = DQ_RB + 2 * 256;                // union list u16
+    static constexpr uint32_t DQ_UF = DQ_U + 2 * (kMaxNbBwd + 8);    // membership per entry
+    static constexpr uint32_t DQ_BAR = ((DQ_UF + kMaxNbBwd + 8 + 7) / 8) * 8;
+    static constexpr int kDqBars = 2 * kDqRing + 2 + 2 + 1 + 1 + 1;
+    static constexpr uint32_t DQ_INT = DQ_BAR + 8 * kDqBars;
+    static constexpr uint32_t kDqSmem = DQ_INT + 16 + 1024;
+};
 
+template <int D>
 __global__ void __launch_bounds__(kDqThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
               const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ dout,
@@ -374,11 +395,16 @@ __global__ void __launch_bounds__(kDqThreads, 1)
               const uint16_t *__restrict__ row_idx, const int32_t *__restrict__ row_cnt,
               __nv_bfloat16 *__restrict__ dq, int *__restrict__ status, int nb, int Hp, int Wp,
               int T, float c, float scale, uint32_t wait_limit, int force_timeout) {
+    using L = DqLayout<D>;
+    constexpr int kHalves = L::kHalves, kDqRing = L::kDqRing;
+    constexpr uint32_t kBlockBytes = L::kBlockBytes, kDqSlot = L::kDqSlot;
+    constexpr uint32_t DQ_RB = L::DQ_RB, DQ_U = L::DQ_U, DQ_UF = L::DQ_UF, DQ_BAR = L::DQ_BAR,
+                       DQ_INT = L::DQ_INT;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
     unsigned char *sm = smem_raw + pad;
-    const uint32_t sRing = raw + pad + DQ_RING;
+    const uint32_t sRing = raw + pad + L::DQ_RING;
     uint32_t *rowBits = reinterpret_cast<uint32_t *>(sm + DQ_RB);  // [2][64 words]
     uint16_t *uList = reinterpret_cast<uint16_t *>(sm + DQ_U);
     uint8_t *uFlag = sm + DQ_UF;
@@ -458,10 +484,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const uint32_t dst = sRing + slot * kDqSlot;
             const int y = row_base + uList[t] * kBlk;
             mbar_expect_tx(&kv_full[slot], kDqSlot);
-            tma_load_2d(dst, &tk, &kv_full[slot], 0, y);
-            tma_load_2d(dst + 8192, &tk, &kv_full[slot], 64, y);
-            tma_load_2d(dst + 16384, &tv, &kv_full[slot], 0, y);
-            tma_load_2d(dst + 24576, &tv, &kv_full[slot], 64, y);
+            for (int h = 0; h < kHalves; ++h) {  // [K halves][V halves], 8 KB each
+                tma_load_2d(dst + h * 8192, &tk, &kv_full[slot], 64 * h, y);
+                tma_load_2d(dst + kBlockBytes + h * 8192, &tv, &kv_full[slot], 64 * h, y);
+            }
         }
         // drain: never leave with a copy in flight
         for (int u = t > kDqRing ? t - kDqRing : 0; u < t; ++u)
@@ -469,7 +495,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer (whole warp, one elected lane issues) ----------------
         constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // Q . K^T, dO . V^T
-        constexpr uint32_t kIdQ = idesc_bf16(128, 128, 0, 1);   // dS . K (K MN-major)
+        constexpr uint32_t kIdQ = idesc_bf16(128, D, 0, 1);     // dS . K (K MN-major)
         auto SdP = [&](int t) -> bool {
             const int slot = t % kDqRing;
             if (!warp_wait(&kv_full[slot], (t / kDqRing) & 1, abort_flag, status, wait_limit))
@@ -478,11 +504,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const uint32_t b0 = sRing + slot * kDqSlot;
             const uint32_t d = tmem + (t & 1) * 128;
 #pragma unroll
-            for (int kk = 0; kk < kD / 16; ++kk) {
+            for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
                 mma_ts_warp(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
-                mma_ts_warp(d + 64, tmem + kColDO + 8 * kk, desc_sw128(b0 + 16384 + off, 16, 1024),
-                       kIdS, kk > 0);
+                mma_ts_warp(d + 64, tmem + kColDO + 8 * kk,
+                            desc_sw128(b0 + kBlockBytes + off, 16, 1024), kIdS, kk > 0);
             }
             mma_commit_warp(&s_full[t & 1]);
             return true;
@@ -524,10 +550,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
         {
             // Q (group 0) or dO (group 1) row -> TMEM, the A operands of S and dP
-            const uint4 *src = reinterpret_cast<const uint4 *>((kg ? dout : q) + grow * kD);
+            const uint4 *src = reinterpret_cast<const uint4 *>((kg ? dout : q) + grow * D);
             const uint32_t col = kg ? kColDO : kColQ;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            for (int half = 0; half < D / 64; ++half) {
                 uint32_t v32[32];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
@@ -575,7 +601,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&ds_full[t & 1]);
         }
-        // ---------------- epilogue: group kg writes dQ features [64 kg, 64 kg + 64) ----------------
+        // ---------------- epilogue: group kg writes dQ features [D/2 kg, D/2 kg + D/2) ----------------
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
         // warp-uniform flags around the collective TMEM loads
@@ -583,12 +609,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         const bool have = (h == 0 || iB >= 0) && !aborted;
         const bool live = have && ntiles > 0 && __all_sync(0xffffffffu, ok);
         if (have) {
-            __nv_bfloat16 *dst = dq + grow * kD + 64 * kg;
+            __nv_bfloat16 *dst = dq + grow * D + (D / 2) * kg;
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
+            for (int part = 0; part < D / 64; ++part) {
                 float v[32];
                 if (live) {
-                    tmem_ld32(tmem + lane_base + kColDQ + 64 * kg + 32 * part, v);
+                    tmem_ld32(tmem + lane_base + kColDQ + (D / 2) * kg + 32 * part, v);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
@@ -614,42 +640,62 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 }  // namespace bwd100
 }  // namespace nabla
 
-cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
-                                        const void *q, const void *k, const void *v,
-                                        const void *o, const void *dout, const float *lse,
-                                        const uint16_t *row_idx, const int32_t *row_cnt,
-                                        const uint16_t *col_idx, const int32_t *col_cnt,
-                                        void *dq, void *dk, void *dv, float *dl, float *l2,
-                                        int *status, int force_timeout, cudaStream_t stream) {
+bool nabla_make_tmap_rows(CUtensorMap *m, const void *base, uint64_t rows, int D);
+
+template <int D>
+static cudaError_t launch_bwd(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
+                              const void *q, const void *k, const void *v, const void *o,
+                              const void *dout, const float *lse, const uint16_t *row_idx,
+                              const int32_t *row_cnt, const uint16_t *col_idx,
+                              const int32_t *col_cnt, void *dq, void *dk, void *dv, float *dl,
+                              float *l2, int *status, int force_timeout, cudaStream_t stream) {
     using namespace nabla::bwd100;
+    constexpr uint32_t kKvSmem = KvLayout<D>::kKvSmem, kDqSmem = DqLayout<D>::kDqSmem;
     const int64_t rows = BH * static_cast<int64_t>(nb) * nabla::kBlk;
     if (rows >= (1ll << 31) || nb > kMaxNbBwd) return cudaErrorInvalidValue;
-    pre_kernel<<<static_cast<unsigned>((rows * 16 + 255) / 256), 256, 0, stream>>>(
+    pre_kernel<D><<<static_cast<unsigned>((rows * (D / 8) + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), lse, dl,
         l2, rows);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     CUtensorMap mq, mk, mv, mdo;
-    if (!nabla_make_tmap_rows128(&mq, q, rows) || !nabla_make_tmap_rows128(&mk, k, rows) ||
-        !nabla_make_tmap_rows128(&mv, v, rows) || !nabla_make_tmap_rows128(&mdo, dout, rows))
+    if (!nabla_make_tmap_rows(&mq, q, rows, D) || !nabla_make_tmap_rows(&mk, k, rows, D) ||
+        !nabla_make_tmap_rows(&mv, v, rows, D) || !nabla_make_tmap_rows(&mdo, dout, rows, D))
         return cudaErrorInvalidValue;
     const float c = scale * 1.4426950408889634f;
     const uint32_t limit = 1000000000u;  // 1 s per wait
-    err = cudaFuncSetAttribute(dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kKvSmem));
     if (err != cudaSuccess) return err;
     const int64_t groups = static_cast<int64_t>((T + 1) / 2) * Hp * Wp;
-    dkdv_kernel<<<static_cast<unsigned>(BH * groups), kKvThreads, kKvSmem, stream>>>(
+    dkdv_kernel<D><<<static_cast<unsigned>(BH * groups), kKvThreads, kKvSmem, stream>>>(
         mq, mk, mv, mdo, l2, dl, col_idx, col_cnt, static_cast<__nv_bfloat16 *>(dk),
         static_cast<__nv_bfloat16 *>(dv), status, nb, Hp, Wp, T, c, scale, limit, force_timeout);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
-    err = cudaFuncSetAttribute(dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kDqSmem));
     if (err != cudaSuccess) return err;
-    dq_kernel<<<static_cast<unsigned>(BH * groups), kDqThreads, kDqSmem, stream>>>(
+    dq_kernel<D><<<static_cast<unsigned>(BH * groups), kDqThreads, kDqSmem, stream>>>(
         mk, mv, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(dout),
         l2, dl, row_idx, row_cnt, static_cast<__nv_bfloat16 *>(dq), status, nb, Hp, Wp, T, c,
         scale, limit, force_timeout);
     return cudaGetLastError();
+}
+
+cudaError_t nabla_launch_attn_bwd_sm100(int64_t BH, int nb, int D, int Hp, int Wp, int T,
+                                        float scale, const void *q, const void *k, const void *v,
+                                        const void *o, const void *dout, const float *lse,
+                                        const uint16_t *row_idx, const int32_t *row_cnt,
+                                        const uint16_t *col_idx, const int32_t *col_cnt,
+                                        void *dq, void *dk, void *dv, float *dl, float *l2,
+                                        int *status, int force_timeout, cudaStream_t stream) {
+    if (D == 128)
+        return launch_bwd<128>(BH, nb, Hp, Wp, T, scale, q, k, v, o, dout, lse, row_idx, row_cnt,
+                               col_idx, col_cnt, dq, dk, dv, dl, l2, status, force_timeout,
+                               stream);
+    if (D == 64)
+        return launch_bwd<64>(BH, nb, Hp, Wp, T, scale, q, k, v, o, dout, lse, row_idx, row_cnt,
+                              col_idx, col_cnt, dq, dk, dv, dl, l2, status, force_timeout, stream);
+    return cudaErrorInvalidValue;
 }

@@ -1,5 +1,5 @@
 // Block-sparse attention forward on 5th-generation tensor cores (tcgen05,
-// TMEM, TMA), head dim 128.
+// TMEM, TMA), head dim D = 128 or 64 (one template).
 //
 // "NABLA: Neighborhood Adaptive Block-Level Attention", section 手法: NABLA,
 // bullet "拡張": attention is computed exactly on the kept 64 x 64 blocks.
@@ -31,9 +31,11 @@
 // threads issues the MMAs (S(t+1) before O += P(t) V(t), so the next scores
 // are computed while this tile's softmax runs); warps 2-9 are the softmax
 // warpgroups (warp w serves TMEM lane quarter w % 4 and key half (w - 2) / 4).
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,384), Q [384,448).  Key half
-// g of a tile has its scores in columns [64 g, 64 g + 64) of the S buffer and
-// its bf16 P in the first 32 of them.
+// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256 + D), Q [384, 384 + D/2).
+// Key half g of a tile has its scores in columns [64 g, 64 g + 64) of the S
+// buffer and its bf16 P in the first 32 of them.  A ring slot holds the two
+// key blocks of a tile for each 64-feature half of D: [half h][block][64 x 64]
+// bf16 at 16 KB per half (one 128-byte swizzle atom wide).
 // Every wait is bounded: on expiry the CTA records a timeout in the status
 // word, unwinds without further work, drains its in-flight copies and MMAs
 // and frees TMEM; later CTAs of the launch see the status and do nothing.
@@ -45,36 +47,45 @@ namespace fwd100 {
 using namespace sm100;
 
 constexpr int kThreads = 320;
-constexpr int kRing = 6;
-constexpr uint32_t kTileBytes = 32768;  // 128 rows x 128 bf16
-constexpr int kD = 128;
 constexpr int kMaxNbFwd = 2048;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleAt = 8.f;  // log2 headroom before a row is rescaled
 constexpr uint32_t kColO = 256, kColQ = 384;
 
-// shared memory map (offsets from a 1024-byte aligned base)
-constexpr uint32_t OFF_RING = 0;                                  // kRing x 32 KB
-constexpr uint32_t OFF_U = OFF_RING + kRing * kTileBytes;         // union list u16
-constexpr uint32_t OFF_UF = OFF_U + 2 * (kMaxNbFwd + 8);          // membership per entry
-constexpr uint32_t OFF_TM = OFF_UF + kMaxNbFwd + 8;               // membership per tile
-// [3][2][128] f32: partial row maxima by tile parity, then the partial sums
-constexpr uint32_t OFF_RED = ((OFF_TM + kMaxNbFwd / 2 + 8 + 15) / 16) * 16;
-constexpr uint32_t OFF_BAR = OFF_RED + 3 * 2 * 128 * 4;
-constexpr int kNumBars = 2 * kRing + 2 + 1 + 2 + 1 + 1 + 1;
-constexpr uint32_t OFF_INT = OFF_BAR + 8 * kNumBars;              // ints
-constexpr uint32_t kSmemBytes = OFF_INT + 16 + 1024;              // + alignment slack
+// shared memory map (offsets from a 1024-byte aligned base) for head dim D
+template <int D>
+struct Layout {
+    static constexpr int kHalves = D / 64;                           // 64-feature halves
+    static constexpr int kRing = D == 128 ? 6 : 10;                  // K/V tiles in flight
+    static constexpr uint32_t kTileBytes = 128u * D * 2;             // 128 rows x D bf16
+    static constexpr uint32_t OFF_RING = 0;
+    static constexpr uint32_t OFF_U = OFF_RING + kRing * kTileBytes;  // union list u16
+    static constexpr uint32_t OFF_UF = OFF_U + 2 * (kMaxNbFwd + 8);   // membership per entry
+    static constexpr uint32_t OFF_TM = OFF_UF + kMaxNbFwd + 8;        // membership per tile
+    // [3][2][128] f32: partial row maxima by tile parity, then the partial sums
+    static constexpr uint32_t OFF_RED = ((OFF_TM + kMaxNbFwd / 2 + 8 + 15) / 16) * 16;
+    static constexpr uint32_t OFF_BAR = OFF_RED + 3 * 2 * 128 * 4;
+    static constexpr int kNumBars = 2 * kRing + 2 + 1 + 2 + 1 + 1 + 1;
+    static constexpr uint32_t OFF_INT = OFF_BAR + 8 * kNumBars;       // ints
+    static constexpr uint32_t kSmemBytes = OFF_INT + 16 + 1024;       // + alignment slack
+};
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                const __nv_bfloat16 *__restrict__ q, const uint32_t *__restrict__ bits,
                __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, int *__restrict__ status,
                int nb, int Hp, int Wp, int T, float c, uint32_t wait_limit, int force_timeout) {
+    using L = Layout<D>;
+    constexpr int kRing = L::kRing, kHalves = L::kHalves;
+    constexpr uint32_t kTileBytes = L::kTileBytes;
+    constexpr uint32_t OFF_U = L::OFF_U, OFF_UF = L::OFF_UF, OFF_TM = L::OFF_TM,
+                       OFF_RED = L::OFF_RED, OFF_BAR = L::OFF_BAR, OFF_INT = L::OFF_INT;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t pad = ((raw + 1023u) & ~1023u) - raw;
     unsigned char *sm = smem_raw + pad;
-    const uint32_t sRing = raw + pad + OFF_RING;
+    const uint32_t sRing = raw + pad + L::OFF_RING;
     uint16_t *uList = reinterpret_cast<uint16_t *>(sm + OFF_U);
     uint8_t *uFlag = sm + OFF_UF;
     uint8_t *tileMem = sm + OFF_TM;
@@ -154,10 +165,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_expect_tx(&kv_full[slot], kTileBytes);
             const int y0 = row_base + uList[2 * t] * kBlk, y1 = row_base + uList[2 * t + 1] * kBlk;
             const uint32_t dst = sRing + slot * kTileBytes;
-            tma_load_2d(dst, tm, &kv_full[slot], 0, y0);
-            tma_load_2d(dst + 8192, tm, &kv_full[slot], 0, y1);
-            tma_load_2d(dst + 16384, tm, &kv_full[slot], 64, y0);
-            tma_load_2d(dst + 24576, tm, &kv_full[slot], 64, y1);
+#pragma unroll
+            for (int h = 0; h < kHalves; ++h) {
+                tma_load_2d(dst + h * 16384, tm, &kv_full[slot], 64 * h, y0);
+                tma_load_2d(dst + h * 16384 + 8192, tm, &kv_full[slot], 64 * h, y1);
+            }
             ++seq;
             return true;
         };
@@ -173,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- MMA issuer (one thread) ----------------
         if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16(128, 128, 0, 0);   // Q . K^T
-            constexpr uint32_t kIdPV = idesc_bf16(128, 128, 0, 1);  // P . V (V MN-major)
+            constexpr uint32_t kIdPV = idesc_bf16(128, D, 0, 1);    // P . V (V MN-major)
             uint32_t seq = 0;
             auto S = [&](int t) -> bool {
                 const int slot = static_cast<int>(seq % kRing);
@@ -183,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t b0 = sRing + slot * kTileBytes;
                 const uint32_t d = tmem + (t & 1) * 128;
 #pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk)
+                for (int kk = 0; kk < D / 16; ++kk)
                     mma_ts_1(d, tmem + kColQ + 8 * kk,
                              desc_sw128(b0 + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), kIdS,
                              kk > 0);
@@ -232,18 +244,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
         {
-            // features [64 g, 64 g + 64) of the Q row -> TMEM (the A operand of S = Q K^T)
-            const uint4 *src = reinterpret_cast<const uint4 *>(q + grow * kD + 64 * g);
-            uint32_t qv[32];
+            // features [D/2 g, D/2 g + D/2) of the Q row -> TMEM columns
+            // [D/4 g, D/4 g + D/4) of Q (the A operand of S = Q K^T)
+            const uint4 *src = reinterpret_cast<const uint4 *>(q + grow * D + (D / 2) * g);
+            uint32_t qv[D / 4];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
+            for (int e = 0; e < D / 16; ++e) {
                 const uint4 v = __ldg(src + e);
                 qv[4 * e] = v.x;
                 qv[4 * e + 1] = v.y;
                 qv[4 * e + 2] = v.z;
                 qv[4 * e + 3] = v.w;
             }
-            tmem_st32(tmem + lane_base + kColQ + 32 * g, reinterpret_cast<float *>(qv));
+            if constexpr (D == 128)
+                tmem_st32(tmem + lane_base + kColQ + 32 * g, reinterpret_cast<float *>(qv));
+            else
+                tmem_st16(tmem + lane_base + kColQ + 16 * g, qv);
             tmem_wait_st();
         }
         tc_fence_before();
@@ -287,13 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = wait_bar(p_empty, (t - 1) & 1, abort_flag, status, wait_limit) && ok;
                     tc_fence_after();
 #pragma unroll
-                    for (int part = 0; part < 2; ++part) {
+                    for (int part = 0; part < D / 64; ++part) {
                         float ov[32];
-                        tmem_ld32(tmem + lane_base + kColO + 64 * g + 32 * part, ov);
+                        tmem_ld32(tmem + lane_base + kColO + (D / 2) * g + 32 * part, ov);
                         tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-                        tmem_st32(tmem + lane_base + kColO + 64 * g + 32 * part, ov);
+                        tmem_st32(tmem + lane_base + kColO + (D / 2) * g + 32 * part, ov);
                     }
                     tmem_wait_st();
                 }
@@ -327,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[t & 1]);
         }
-        // ---------------- epilogue: half g writes features [64 g, 64 g + 64) ----------------
+        // ---------------- epilogue: half g writes features [D/2 g, D/2 g + D/2) ----------------
         if (ok && ntiles > 0) ok = wait_bar(o_done, 0, abort_flag, status, wait_limit);
         tc_fence_after();
         red[(4 + g) * 128 + r] = l;  // own slot: the partner may still read the last maxima
@@ -342,12 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool live = read_o && l > 0.f;
             if (lse != nullptr && g == 0) lse[grow] = live ? (m + log2f(l)) * kLn2 : -INFINITY;
             const float inv = live ? 1.f / l : 0.f;
-            __nv_bfloat16 *dst = out + grow * kD + 64 * g;
+            __nv_bfloat16 *dst = out + grow * D + (D / 2) * g;
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
+            for (int part = 0; part < D / 64; ++part) {
                 float ov[32];
                 if (read_o) {
-                    tmem_ld32(tmem + lane_base + kColO + 64 * g + 32 * part, ov);
+                    tmem_ld32(tmem + lane_base + kColO + (D / 2) * g + 32 * part, ov);
                     tmem_wait_ld();
                 } else {
 #pragma unroll
@@ -399,12 +415,13 @@ EncodeTiledFn encode_fn() {
 
 }  // namespace
 
-// [rows, 128] bf16 row-major, boxes of 64 rows x 64 features, 128-byte swizzle
-bool nabla_make_tmap_rows128(CUtensorMap *m, const void *base, uint64_t rows) {
+// [rows, D] bf16 row-major (D = 64 or 128), boxes of 64 rows x 64 features,
+// 128-byte swizzle
+bool nabla_make_tmap_rows(CUtensorMap *m, const void *base, uint64_t rows, int D) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
-    const cuuint64_t dims[2] = {128, rows};
-    const cuuint64_t strides[1] = {128 * 2};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
     const cuuint32_t box[2] = {64, 64};
     const cuuint32_t es[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
@@ -412,26 +429,40 @@ bool nabla_make_tmap_rows128(CUtensorMap *m, const void *base, uint64_t rows) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-size_t nabla_fwd_sm100_smem() { return nabla::fwd100::kSmemBytes; }
-
-cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
-                                        const void *q, const void *k, const void *v,
-                                        const uint32_t *bits, void *o, float *lse, int *status,
-                                        int force_timeout, cudaStream_t stream) {
+template <int D>
+static cudaError_t launch_fwd(int64_t BH, int nb, int Hp, int Wp, int T, float scale,
+                              const void *q, const void *k, const void *v, const uint32_t *bits,
+                              void *o, float *lse, int *status, int force_timeout,
+                              cudaStream_t stream) {
     using namespace nabla::fwd100;
+    constexpr uint32_t kSmem = Layout<D>::kSmemBytes;
     const uint64_t rows = static_cast<uint64_t>(BH) * nb * nabla::kBlk;
     if (rows >= (1ull << 31) || nb > kMaxNbFwd) return cudaErrorInvalidValue;
     CUtensorMap mk, mv;
-    if (!nabla_make_tmap_rows128(&mk, k, rows) || !nabla_make_tmap_rows128(&mv, v, rows))
+    if (!nabla_make_tmap_rows(&mk, k, rows, D) || !nabla_make_tmap_rows(&mv, v, rows, D))
         return cudaErrorInvalidValue;
-    cudaError_t err = cudaFuncSetAttribute(fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(kSmemBytes));
+    cudaError_t err = cudaFuncSetAttribute(fwd_kernel<D>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(kSmem));
     if (err != cudaSuccess) return err;
     const int64_t groups = static_cast<int64_t>((T + 1) / 2) * Hp * Wp;
     const float c = scale * 1.4426950408889634f;
     const uint32_t limit = 1000000000u;  // 1 s per wait
-    fwd_kernel<<<static_cast<unsigned>(BH * groups), kThreads, kSmemBytes, stream>>>(
+    fwd_kernel<D><<<static_cast<unsigned>(BH * groups), kThreads, kSmem, stream>>>(
         mk, mv, static_cast<const __nv_bfloat16 *>(q), bits, static_cast<__nv_bfloat16 *>(o), lse,
         status, nb, Hp, Wp, T, c, limit, force_timeout);
     return cudaGetLastError();
+}
+
+cudaError_t nabla_launch_attn_fwd_sm100(int64_t BH, int nb, int D, int Hp, int Wp, int T,
+                                        float scale, const void *q, const void *k, const void *v,
+                                        const uint32_t *bits, void *o, float *lse, int *status,
+                                        int force_timeout, cudaStream_t stream) {
+    if (D == 128)
+        return launch_fwd<128>(BH, nb, Hp, Wp, T, scale, q, k, v, bits, o, lse, status,
+                               force_timeout, stream);
+    if (D == 64)
+        return launch_fwd<64>(BH, nb, Hp, Wp, T, scale, q, k, v, bits, o, lse, status,
+                              force_timeout, stream);
+    return cudaErrorInvalidValue;
 }

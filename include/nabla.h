@@ -65,7 +65,7 @@ typedef struct CUstream_st *nabla_stream_t; /* == cudaStream_t */
  * depends on the scores (0 < p < 1 and not NABLA_FULL_STA). */
 #define NABLA_DEBUG_SCORES 8u
 /* Test aid, not for production: makes the tensor-core attention forward and
- * backward (D = 128) give up a device-side wait at once, so that the timeout
+ * backward give up a device-side wait at once, so that the timeout
  * path (status word = NABLA_ERR_TIMEOUT, clean unwind, context still usable)
  * can be exercised without faulting or hanging the GPU.  Outputs are not
  * meaningful after it. */
@@ -257,7 +257,7 @@ int nabla_build_mask_dr(const nabla_shape *shape, const nabla_dr_params *params,
  *   lse_n = log sum_m exp(scale * q_n . k_m)          (float32 [B*heads, N])
  * Needs mask->bits, mask->row_idx and mask->row_cnt.  lse may be NULL when
  * no backward follows.  Workspace: nabla_workspace_size(shape,
- * NABLA_OP_ATTN_FWD).  D = 128 runs on the tcgen05 tensor cores; a device-side
+ * NABLA_OP_ATTN_FWD).  Runs on the tcgen05 tensor cores; a device-side
  * wait that expires (it never should) is reported through nabla_status() and
  * leaves O and lse unwritten. */
 int nabla_attn_fwd(const nabla_shape *shape, const nabla_params *params, const nabla_bf16 *q,

@@ -85,9 +85,19 @@ def test_tiny_backward():
     _bwd_parity(Case(synth.WORKLOADS["tiny"], backward=True))
 
 
-def test_ragged_backward():
-    w = synth.Workload("odd130b", 1, 2, 5, 16, 104, 128, (2, 4, 4), 0.7, backward=True)
+@pytest.mark.parametrize("D", [128, 64])
+def test_ragged_backward(D):
+    # 130 blocks in 5 frames: the last temporal pair has one member
+    w = synth.Workload("odd130b", 1, 2, 5, 16, 104, D, (2, 4, 4), 0.7, backward=True)
     _bwd_parity(Case(w))
+
+
+def test_ragged_forward_and_backward_d64_wide():
+    # D = 64, 150 blocks in 3 frames of a 5 x 10 patch grid
+    w = synth.Workload("odd150b", 1, 2, 3, 40, 80, 64, (3, 8, 8), 0.9, backward=True)
+    c = Case(w)
+    _fwd_parity(c)
+    _bwd_parity(c)
 
 
 def test_backward_deterministic():
@@ -104,12 +114,13 @@ def test_backward_deterministic():
         assert torch.equal(a, b)
 
 
-def test_forward_timeout_is_reported_and_the_context_survives():
+@pytest.mark.parametrize("D", [128, 64])
+def test_forward_timeout_is_reported_and_the_context_survives(D):
     # The test flag makes the forward's first device-side wait give up at once
     # (a barrier nothing arrives on, with a tiny poll limit): the kernel must
     # record NABLA_ERR_TIMEOUT, unwind and free its resources; the next call
     # on the same context must run normally and be correct.
-    w = synth.Workload("odd130", 2, 2, 5, 16, 104, 128, (2, 4, 4), 0.7)
+    w = synth.Workload("odd130", 2, 2, 5, 16, 104, D, (2, 4, 4), 0.7)
     c = Case(w)
     gm = c.gpu_mask()
     ws = nabla.workspace(c.shape, nabla.OP_ATTN_FWD, "cuda")
@@ -124,12 +135,13 @@ def test_forward_timeout_is_reported_and_the_context_survives():
     assert_close(bf16_to_f64(o).reshape(-1, L, w.D), oo, "O after timeout")
 
 
-def test_backward_timeout_is_reported_and_the_context_survives():
+@pytest.mark.parametrize("D", [128, 64])
+def test_backward_timeout_is_reported_and_the_context_survives(D):
     # As for the forward: the flag makes the backward's first device-side wait
     # (in the dK/dV kernel; the dQ kernel then sees the status and skips) give
     # up at once; the status must read NABLA_ERR_TIMEOUT and the next backward
     # on the same context and workspace must be correct.
-    w = synth.Workload("odd130b", 1, 2, 5, 16, 104, 128, (2, 4, 4), 0.7, backward=True)
+    w = synth.Workload("odd130b", 1, 2, 5, 16, 104, D, (2, 4, 4), 0.7, backward=True)
     c = Case(w)
     gm = c.gpu_mask()
     o, lse = nabla.attn_fwd(c.shape, c.params(), c.gpu["q"], c.gpu["k"], c.gpu["v"], gm)
