@@ -6,7 +6,7 @@
 //                      float32 running sum in ascending token order, * 1/64.
 //                      Q-bar row-major [BH, nb, D]; K-bar transposed
 //                      [BH, D, nb] so the score kernel streams it coalesced.
-//   score_cut_kernel   per (bh, 16 query blocks): pooled scores as a float32
+//   score_cut_kernel   per (bh, 8 query blocks): pooled scores as a float32
 //                      fma chain over d ascending (register-tiled FFMA; the
 //                      order per output is the plain ascending chain), then
 //                      per row (one warp): weights exp(s - max) in float64,
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(256) flatten_pool_kernel(
 // ---------------------------------------------------------------------------
 // scores + CDF cut + STA + lists
 // ---------------------------------------------------------------------------
-constexpr int kRows = 16;       // query blocks per CTA
+constexpr int kRows = 8;        // query blocks per CTA (one per warp)
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 256;          // bins of one row's mass histogram
@@ -303,10 +303,10 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t b, double u) {
     atomicAdd(hist + kBins + b, static_cast<uint32_t>(ui & 0xFFFFFull));
 }
 
-// One CTA per (bh, 16 query blocks).
-//   Phase 1: the 16 x nb pooled scores into shared memory.  Thread t owns
+// One CTA per (bh, 8 query blocks), three CTAs per SM.
+//   Phase 1: the 8 x nb pooled scores into shared memory.  Thread t owns
 //            the column pairs (2t, 2t + 1), (2t + 512, 2t + 513), ...; for each
-//            it runs the 32 fma chains (16 rows x 2 columns) over d = 0 .. D-1
+//            it runs the 16 fma chains (8 rows x 2 columns) over d = 0 .. D-1
 //            as packed fma.rn.f32x2 on row pairs (each lane rounds like fmaf),
 //            the query means broadcast from shared memory and the K-bar^T
 //            column pair read from L2 with 8 features prefetched in registers;
@@ -323,7 +323,7 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t b, double u) {
 //   Then the bit row (adaptive set OR STA window OR diagonal) and its
 //   ascending list are written.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 3)
     score_cut_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar_t,
                      CutParams prm, uint32_t *__restrict__ bits, uint16_t *__restrict__ row_idx,
                      int32_t *__restrict__ row_cnt, float *__restrict__ scores_out) {
