@@ -16,7 +16,8 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, in
                                     const void *q, const void *k, float *qbar, float *kbar_t,
                                     uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
                                     uint16_t *col_idx, int32_t *col_cnt, float *scores,
-                                    cudaStream_t stream, const void *q_grid, const void *k_grid);
+                                    cudaStream_t stream, const void *q_grid, const void *k_grid,
+                                    int *ctr, int *status);
 cudaError_t nabla_launch_build_mask_dr(int64_t BH, int nb, int D, int T, int Hp, int Wp, int mode,
                                        double gamma, double lambda, float tau, float scale, int wt,
                                        int wh, int ww, unsigned flags, const void *q,
@@ -43,7 +44,9 @@ constexpr int kMaxNb = 2048;
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Scratch of the mask build: pooled Q [BH, nb, D] then pooled K transposed
-// [BH, D, nbp] (nbp = nb rounded up to a multiple of 4).
+// [BH, D, nbp] (nbp = nb rounded up to a multiple of 4).  In a workspace they
+// follow the status region and the task counters of the persistent front end
+// (1 + BH ints).
 struct MaskScratch {
     size_t qbar_bytes, kbar_bytes;
 };
@@ -96,10 +99,12 @@ size_t mask_scratch_bytes(const Dims &d) {
     return m.qbar_bytes + m.kbar_bytes;
 }
 
+size_t counter_bytes(const Dims &d) { return round256(sizeof(int) * (1 + d.BH)); }
+
 size_t ws_bytes(const Dims &d, int op) {
     switch (op) {
         case NABLA_OP_BUILD_MASK:
-            return kStatusBytes + mask_scratch_bytes(d);
+            return kStatusBytes + counter_bytes(d) + mask_scratch_bytes(d);
         case NABLA_OP_ATTN_FWD:
             return kStatusBytes;
         case NABLA_OP_ATTN_BWD:  // D_n and lse_n * log2(e)
@@ -199,14 +204,16 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params, const
     if ((st = check_ws(d, NABLA_OP_BUILD_MASK, workspace, workspace_bytes)) != NABLA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
-    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
+    int *ctr = reinterpret_cast<int *>(static_cast<unsigned char *>(workspace) + kStatusBytes);
+    unsigned char *w = reinterpret_cast<unsigned char *>(ctr) + counter_bytes(d);
     float *qbar = reinterpret_cast<float *>(w);
     float *kbar_t = reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
         d.BH, d.nb, d.D, shape->T, d.Hp, d.Wp, params->p, params->scale, params->sta_t,
         params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
         mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
-        cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, nullptr, nullptr));
+        cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, nullptr, nullptr, ctr,
+        static_cast<int *>(workspace)));
 }
 
 int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
@@ -231,14 +238,16 @@ int nabla_build_mask_grid(const nabla_shape *shape, const nabla_params *params,
     if ((st = check_ws(d, NABLA_OP_BUILD_MASK, workspace, workspace_bytes)) != NABLA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
-    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
+    int *ctr = reinterpret_cast<int *>(static_cast<unsigned char *>(workspace) + kStatusBytes);
+    unsigned char *w = reinterpret_cast<unsigned char *>(ctr) + counter_bytes(d);
     float *qbar = reinterpret_cast<float *>(w);
     float *kbar_t = reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes);
     return cuda_status(nabla_launch_build_mask(
         d.BH, d.nb, d.D, shape->T, d.Hp, d.Wp, params->p, params->scale, params->sta_t,
         params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
         mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
-        cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, q_grid, k_grid));
+        cols ? mask->col_cnt : nullptr, debug_scores(params, mask), s, q_grid, k_grid, ctr,
+        static_cast<int *>(workspace)));
 }
 
 int nabla_build_mask_dr(const nabla_shape *shape, const nabla_dr_params *params,
@@ -268,7 +277,7 @@ int nabla_build_mask_dr(const nabla_shape *shape, const nabla_dr_params *params,
     if ((st = check_ws(d, op, workspace, workspace_bytes)) != NABLA_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if ((st = clear_status(workspace, s)) != NABLA_OK) return st;
-    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes;
+    unsigned char *w = static_cast<unsigned char *>(workspace) + kStatusBytes + counter_bytes(d);
     float *qbar = thr ? reinterpret_cast<float *>(w) : nullptr;
     float *kbar_t = thr ? reinterpret_cast<float *>(w + mask_scratch(d).qbar_bytes) : nullptr;
     const bool cols = (params->flags & NABLA_EMIT_COLS) != 0;
@@ -415,5 +424,5 @@ extern "C" int nabla_build_mask_static(const nabla_shape *shape, const nabla_par
         params->sta_h, params->sta_w, params->flags, q, k, qbar, kbar_t, mask->bits,
         mask->row_idx, mask->row_cnt, cols ? mask->col_idx : nullptr,
         cols ? mask->col_cnt : nullptr, debug_scores(params, mask),
-        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr));
+        reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, nullptr));
 }

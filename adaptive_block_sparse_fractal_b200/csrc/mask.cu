@@ -21,6 +21,8 @@
 //
 // The mass sums are exact integers, so the selected set does not depend on
 // the order in which threads add them.
+#include <algorithm>
+
 #include "common.cuh"
 #include "exp_nonpos.cuh"
 
@@ -29,21 +31,21 @@ namespace nabla {
 // ---------------------------------------------------------------------------
 // pooling
 // ---------------------------------------------------------------------------
-// CTA = 256 threads = (256 / CH) blocks x CH chunks of 8 features, CH = D/8.
+// A tile = 256 threads = (256 / CH) blocks x CH chunks of 8 features,
+// CH = D/8; tile index cta = which * BH * tiles + bh * tiles + tile (which 0:
+// Q, 1: K).  `tile` is [256 / CH][D + 1] floats of shared memory.
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restrict__ q,
-                                                   const __nv_bfloat16 *__restrict__ k,
-                                                   float *__restrict__ qbar,
-                                                   float *__restrict__ kbar_t, int64_t BH,
-                                                   int nb) {
+__device__ __forceinline__ void pool_tile(const __nv_bfloat16 *__restrict__ q,
+                                          const __nv_bfloat16 *__restrict__ k,
+                                          float *__restrict__ qbar, float *__restrict__ kbar_t,
+                                          int64_t BH, int nb, int64_t cta,
+                                          float (*tile)[D + 1]) {
     constexpr int CH = D / 8;
-    constexpr int BPC = 256 / CH;  // blocks per CTA
-    __shared__ float tile[BPC][D + 1];
+    constexpr int BPC = 256 / CH;  // blocks per tile
     const int tid = threadIdx.x;
     const int c = tid % CH;
     const int bl = tid / CH;
     const int tiles_per_head = (nb + BPC - 1) / BPC;
-    const int64_t cta = blockIdx.x;
     const int which = static_cast<int>(cta / (BH * tiles_per_head));  // 0: q, 1: k
     const int64_t rem = cta % (BH * tiles_per_head);
     const int64_t bh = rem / tiles_per_head;
@@ -101,6 +103,16 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restri
     }
 }
 
+template <int D>
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restrict__ q,
+                                                   const __nv_bfloat16 *__restrict__ k,
+                                                   float *__restrict__ qbar,
+                                                   float *__restrict__ kbar_t, int64_t BH,
+                                                   int nb) {
+    __shared__ float tile[256 / (D / 8)][D + 1];
+    pool_tile<D>(q, k, qbar, kbar_t, BH, nb, blockIdx.x, tile);
+}
+
 // ---------------------------------------------------------------------------
 // fused flatten + pooling: reads Q or K in GRID order [B*h, T, H, W, D], writes
 // the flattened copy [B*h, N, D] and the pooled block means in one pass.
@@ -110,19 +122,18 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16 *__restri
 // paths give the same bits.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) flatten_pool_kernel(
+__device__ __forceinline__ void flatten_pool_tile(
     const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
     __nv_bfloat16 *__restrict__ qf, __nv_bfloat16 *__restrict__ kf, float *__restrict__ qbar,
-    float *__restrict__ kbar_t, int64_t BH, int nb, int H, int W) {
+    float *__restrict__ kbar_t, int64_t BH, int nb, int H, int W, int64_t cta,
+    float (*tile)[D + 1]) {
     constexpr int CH = D / 8;
-    constexpr int BPC = 256 / CH;  // blocks per CTA
+    constexpr int BPC = 256 / CH;  // blocks per tile
     constexpr int P = 8;
-    __shared__ float tile[BPC][D + 1];
     const int tid = threadIdx.x;
     const int c = tid % CH;
     const int bl = tid / CH;
     const int tiles_per_head = (nb + BPC - 1) / BPC;
-    const int64_t cta = blockIdx.x;
     const int which = static_cast<int>(cta / (BH * tiles_per_head));  // 0: q, 1: k
     const int64_t rem = cta % (BH * tiles_per_head);
     const int64_t bh = rem / tiles_per_head;
@@ -186,6 +197,15 @@ __global__ void __launch_bounds__(256) flatten_pool_kernel(
             }
         }
     }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) flatten_pool_kernel(
+    const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+    __nv_bfloat16 *__restrict__ qf, __nv_bfloat16 *__restrict__ kf, float *__restrict__ qbar,
+    float *__restrict__ kbar_t, int64_t BH, int nb, int H, int W) {
+    __shared__ float tile[256 / (D / 8)][D + 1];
+    flatten_pool_tile<D>(q, k, qf, kf, qbar, kbar_t, BH, nb, H, W, blockIdx.x, tile);
 }
 
 // ---------------------------------------------------------------------------
@@ -322,12 +342,17 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t b, double u) {
 //            split are resolved by score group, lowest index first.)
 //   Then the bit row (adaptive set OR STA window OR diagonal) and its
 //   ascending list are written.
+// Rows [i0, i0 + 8) of head bh; `smem` is nabla_score_cut_smem() bytes.  The
+// pooled means are read through L2 (ld.global.cg), so a tile may run in the
+// same launch that wrote them.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 3)
-    score_cut_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar_t,
-                     CutParams prm, uint32_t *__restrict__ bits, uint16_t *__restrict__ row_idx,
-                     int32_t *__restrict__ row_cnt, float *__restrict__ scores_out) {
-    extern __shared__ __align__(16) unsigned char smem[];
+__device__ __forceinline__ void score_cut_tile(const float *__restrict__ qbar,
+                                               const float *__restrict__ kbar_t,
+                                               const CutParams &prm, uint32_t *__restrict__ bits,
+                                               uint16_t *__restrict__ row_idx,
+                                               int32_t *__restrict__ row_cnt,
+                                               float *__restrict__ scores_out, int64_t bh, int i0,
+                                               unsigned char *smem) {
     const int nb = prm.nb;
     const int nbp = (nb + 3) & ~3;
     float *sS = reinterpret_cast<float *>(smem);                  // [kRows][nbp]
@@ -337,15 +362,12 @@ __global__ void __launch_bounds__(kThreads, 3)
     int *sE = reinterpret_cast<int *>(sW + kWarps * kMaxWords);   // [kWarps][kCand]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int tiles = (nb + kRows - 1) / kRows;
-    const int64_t bh = blockIdx.x / tiles;
-    const int i0 = (blockIdx.x % tiles) * kRows;
     const int rows_here = min(kRows, nb - i0);
 
     // ---- phase 1
     for (int idx = tid; idx < kRows * D; idx += kThreads) {
         const int r = idx / D, d = idx % D;
-        sQt[d * kRows + r] = (r < rows_here) ? qbar[(bh * nb + i0 + r) * D + d] : 0.f;
+        sQt[d * kRows + r] = (r < rows_here) ? __ldcg(qbar + (bh * nb + i0 + r) * D + d) : 0.f;
     }
     __syncthreads();
     const float *kt = kbar_t + bh * static_cast<int64_t>(D) * nbp;
@@ -360,13 +382,13 @@ __global__ void __launch_bounds__(kThreads, 3)
         float2 kc[kPre], kn[kPre];
 #pragma unroll
         for (int q = 0; q < kPre; ++q)
-            kc[q] = __ldg(reinterpret_cast<const float2 *>(kt + static_cast<int64_t>(q) * nbp + j));
+            kc[q] = __ldcg(reinterpret_cast<const float2 *>(kt + static_cast<int64_t>(q) * nbp + j));
 #pragma unroll
         for (int d0 = 0; d0 < D; d0 += kPre) {
             if (d0 + kPre < D) {
 #pragma unroll
                 for (int q = 0; q < kPre; ++q)
-                    kn[q] = __ldg(reinterpret_cast<const float2 *>(
+                    kn[q] = __ldcg(reinterpret_cast<const float2 *>(
                         kt + static_cast<int64_t>(d0 + kPre + q) * nbp + j));
             }
 #pragma unroll
@@ -649,6 +671,122 @@ __global__ void __launch_bounds__(kThreads, 3)
     }
 }
 
+template <int D>
+__global__ void __launch_bounds__(kThreads, 3)
+    score_cut_kernel(const float *__restrict__ qbar, const float *__restrict__ kbar_t,
+                     CutParams prm, uint32_t *__restrict__ bits, uint16_t *__restrict__ row_idx,
+                     int32_t *__restrict__ row_cnt, float *__restrict__ scores_out) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int tiles = (prm.nb + kRows - 1) / kRows;
+    score_cut_tile<D>(qbar, kbar_t, prm, bits, row_idx, row_cnt, scores_out, blockIdx.x / tiles,
+                      static_cast<int>(blockIdx.x % tiles) * kRows, smem);
+}
+
+// ---------------------------------------------------------------------------
+// Persistent front end: the pooling (or flattening + pooling) tiles and the
+// score/cut tiles of every head in one launch, so that the HBM-bound pooling
+// of head h + 1 runs beside the issue-bound scores and cut of head h.  CTAs
+// take tasks in order from a counter: the pooling tiles of head 0, then for
+// h = 1 .. BH the pooling tiles of head h (while h < BH) followed by the
+// score/cut tiles of head h - 1.  A score/cut tile waits until its head's
+// pooling tiles have all finished (a per-head counter; every pooling tile it
+// needs was taken earlier by a running CTA that never waits, so the wait
+// always ends); the wait is bounded (1 s of %globaltimer), after which the
+// status word records a timeout and the remaining score/cut tiles are
+// skipped.  ctr[0] = next task, ctr[1 + bh] = finished pooling tiles of head
+// bh, all zero at launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+template <int D, bool kGrid>
+__global__ void __launch_bounds__(kThreads, 3)
+    front_kernel(const __nv_bfloat16 *__restrict__ q_grid, const __nv_bfloat16 *__restrict__ k_grid,
+                 const __nv_bfloat16 *q, const __nv_bfloat16 *k, float *qbar, float *kbar_t,
+                 CutParams prm, uint32_t *__restrict__ bits, uint16_t *__restrict__ row_idx,
+                 int32_t *__restrict__ row_cnt, float *__restrict__ scores_out, int *ctr,
+                 int *status, int64_t BH, int H, int W) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    __shared__ int s_task, s_go;
+    constexpr int BPC = 256 / (D / 8);
+    const int nb = prm.nb;
+    const int tiles = (nb + BPC - 1) / BPC;
+    const int P = 2 * tiles;                    // pooling tiles per head (Q and K)
+    const int S = (nb + kRows - 1) / kRows;     // score/cut tiles per head
+    const int64_t total = BH * static_cast<int64_t>(P + S);
+    float(*tile)[D + 1] = reinterpret_cast<float(*)[D + 1]>(smem);
+    for (;;) {
+        __syncthreads();  // the previous task is done with shared memory
+        if (threadIdx.x == 0) s_task = atomicAdd(ctr, 1);
+        __syncthreads();
+        const int64_t t = s_task;
+        if (t >= total) break;
+        // decode: [P pool(0)] [P pool(1), S score(0)] ... [P pool(BH-1), S score(BH-2)] [S score(BH-1)]
+        bool pool;
+        int64_t bh;
+        int idx;
+        if (t < P) {
+            pool = true, bh = 0, idx = static_cast<int>(t);
+        } else {
+            const int64_t u = t - P, blk = u / (P + S);
+            const int r = static_cast<int>(u % (P + S));
+            if (blk + 1 < BH) {
+                pool = r < P;
+                bh = pool ? blk + 1 : blk;
+                idx = pool ? r : r - P;
+            } else {
+                pool = false, bh = BH - 1, idx = static_cast<int>(u - (BH - 1) * (P + S));
+            }
+        }
+        if (pool) {
+            const int64_t cta = (idx / tiles) * BH * tiles + bh * tiles + idx % tiles;
+            if (kGrid)
+                flatten_pool_tile<D>(q_grid, k_grid, const_cast<__nv_bfloat16 *>(q),
+                                     const_cast<__nv_bfloat16 *>(k), qbar, kbar_t, BH, nb, H, W,
+                                     cta, tile);
+            else
+                pool_tile<D>(q, k, qbar, kbar_t, BH, nb, cta, tile);
+            __threadfence();  // this thread's pooled means, visible GPU-wide
+            __syncthreads();
+            if (threadIdx.x == 0) atomicAdd(ctr + 1 + bh, 1);
+        } else {
+            if (threadIdx.x == 0) {
+                // the test aid NABLA_DEBUG_TIMEOUT waits for one pooling tile
+                // too many, with a 1 ms limit: the wait must run out
+                const bool test_wait = (prm.flags & 0x100u) != 0;
+                const int need = test_wait ? P + 1 : P;
+                const uint64_t limit = test_wait ? 1000000ull : 1000000000ull;
+                int go = *reinterpret_cast<volatile int *>(status) == kDevOk;
+                if (go && ld_acquire_gpu(ctr + 1 + bh) < need) {
+                    const uint64_t t0 = global_ns();
+                    for (int n = 0; ld_acquire_gpu(ctr + 1 + bh) < need; ++n) {
+                        if (global_ns() - t0 > limit) {  // give up
+                            atomicExch(status, kDevTimeout);
+                            go = 0;
+                            break;
+                        }
+                        if (n > 64) __nanosleep(128);
+                    }
+                }
+                s_go = go;
+            }
+            __syncthreads();
+            if (s_go)
+                score_cut_tile<D>(qbar, kbar_t, prm, bits, row_idx, row_cnt, scores_out, bh,
+                                  idx * kRows, smem);
+        }
+    }
+}
+
 // (frame, patch row, patch column) of block j, advanced by a fixed stride
 // without integer division (the emit loop visits j = lane, lane + 32, ...).
 struct BlockCoord {
@@ -860,17 +998,77 @@ static cudaError_t launch_score_cut(dim3 grid, size_t smem, const float *qbar,
     return cudaGetLastError();
 }
 
+template <int D, bool kGrid>
+static cudaError_t launch_front(const void *q_grid, const void *k_grid, const void *q,
+                                const void *k, float *qbar, float *kbar_t, nabla::CutParams prm,
+                                uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
+                                float *scores, int *ctr, int *status, int64_t BH, int H, int W,
+                                cudaStream_t stream) {
+    using namespace nabla;
+    auto kern = front_kernel<D, kGrid>;
+    const size_t smem = nabla_score_cut_smem(prm.nb, D);
+    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    err = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (err != cudaSuccess) return err;
+    int dev = 0, sms = 0, per_sm = 0;
+    if ((err = cudaGetDevice(&dev)) != cudaSuccess) return err;
+    if ((err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return err;
+    if ((err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem)) !=
+        cudaSuccess)
+        return err;
+    const int bpc = 256 / (D / 8);
+    const int64_t tasks =
+        BH * (2 * ((prm.nb + bpc - 1) / bpc) + (prm.nb + kRows - 1) / kRows);
+    const int64_t grid = std::min<int64_t>(tasks, static_cast<int64_t>(sms) * std::max(per_sm, 1));
+    if ((err = cudaMemsetAsync(ctr, 0, sizeof(int) * (1 + BH), stream)) != cudaSuccess) return err;
+    kern<<<static_cast<unsigned>(grid), kThreads, smem, stream>>>(
+        static_cast<const __nv_bfloat16 *>(q_grid), static_cast<const __nv_bfloat16 *>(k_grid),
+        static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), qbar, kbar_t,
+        prm, bits, row_idx, row_cnt, scores, ctr, status, BH, H, W);
+    return cudaGetLastError();
+}
+
 // q_grid/k_grid non-null: q and k are in grid order; flatten them into q/k
 // (then outputs) in the same pass as the pooling.  scores non-null: also
 // write the pooled scores [BH, nb, nb] (only when the mask depends on them).
+// ctr non-null with grid-order inputs (1 + BH ints of device memory, cleared
+// here): the flattening + pooling and the scores and cut run in one
+// persistent launch; otherwise as a pooling launch followed by a score/cut
+// launch.
 cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, int Wp, float p,
                                     float scale, int wt, int wh, int ww, unsigned flags,
                                     const void *q, const void *k, float *qbar, float *kbar_t,
                                     uint32_t *bits, uint16_t *row_idx, int32_t *row_cnt,
                                     uint16_t *col_idx, int32_t *col_cnt, float *scores,
-                                    cudaStream_t stream, const void *q_grid, const void *k_grid) {
+                                    cudaStream_t stream, const void *q_grid, const void *k_grid,
+                                    int *ctr, int *status) {
     using namespace nabla;
     CutParams prm{nb, T, Hp, Wp, wt, wh, ww, flags, p, scale, 0, 0.f};
+    const bool score_free = p <= 0.0f || p >= 1.0f || (flags & 2u);
+    if (ctr != nullptr && q_grid != nullptr && !score_free) {
+        // flattening + pooling (HBM-bound, 2 x 2 bytes per element moved) beside
+        // the scores and cut in one persistent launch.  (From already
+        // flattened inputs the pooling is too short to gain from it: measured
+        // no faster, so that case keeps the two launches below.)
+        cudaError_t err =
+            D == 128 ? launch_front<128, true>(q_grid, k_grid, q, k, qbar, kbar_t, prm, bits,
+                                               row_idx, row_cnt, scores, ctr, status, BH, Hp * 8,
+                                               Wp * 8, stream)
+                     : launch_front<64, true>(q_grid, k_grid, q, k, qbar, kbar_t, prm, bits,
+                                              row_idx, row_cnt, scores, ctr, status, BH, Hp * 8,
+                                              Wp * 8, stream);
+        if (err != cudaSuccess) return err;
+        if (col_idx) {
+            const int words = (nb + 31) / 32;
+            col_lists_kernel<<<static_cast<unsigned>(BH * words), kColWarps * 32, 0, stream>>>(
+                bits, col_idx, col_cnt, nb);
+            err = cudaGetLastError();
+        }
+        return err;
+    }
     cudaError_t err;
     const bool from_grid = q_grid != nullptr;
     const int bpc = 256 / (D / 8);
@@ -893,7 +1091,7 @@ cudaError_t nabla_launch_build_mask(int64_t BH, int nb, int D, int T, int Hp, in
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
-    if (p <= 0.0f || p >= 1.0f || (flags & 2u)) {
+    if (score_free) {
         // the mask does not depend on the scores
         const int64_t rows = BH * nb;
         sta_emit_kernel<<<static_cast<unsigned>((rows * 32 + 255) / 256), 256, 0, stream>>>(
@@ -944,7 +1142,7 @@ cudaError_t nabla_launch_build_mask_dr(int64_t BH, int nb, int D, int T, int Hp,
                                        int32_t *col_cnt, float *scores, cudaStream_t stream) {
     using namespace nabla;
     CutParams prm{nb, T, Hp, Wp, wt, wh, ww, flags, 1.0f, scale, mode, tau};
-    cudaError_t err;
+    cudaError_t err = cudaSuccess;
     const int words = (nb + 31) / 32;
     const dim3 col_grid(static_cast<unsigned>(BH * words));
     if (flags & 2u) {  // the full window: every block

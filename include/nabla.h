@@ -65,10 +65,11 @@ typedef struct CUstream_st *nabla_stream_t; /* == cudaStream_t */
  * depends on the scores (0 < p < 1 and not NABLA_FULL_STA). */
 #define NABLA_DEBUG_SCORES 8u
 /* Test aid, not for production: makes the tensor-core attention forward and
- * backward give up a device-side wait at once, so that the timeout
- * path (status word = NABLA_ERR_TIMEOUT, clean unwind, context still usable)
- * can be exercised without faulting or hanging the GPU.  Outputs are not
- * meaningful after it. */
+ * backward, and the persistent front end of nabla_build_mask_grid, give up a
+ * device-side wait at once (or after 1 ms), so that the timeout path (status
+ * word = NABLA_ERR_TIMEOUT, clean unwind, context still usable) can be
+ * exercised without faulting or hanging the GPU.  Outputs are not meaningful
+ * after it. */
 #define NABLA_DEBUG_TIMEOUT 0x100u
 
 /* Problem shape.  P must be 8. */
@@ -175,7 +176,10 @@ int nabla_build_mask(const nabla_shape *shape, const nabla_params *params,
  * "トークン再順序付け (Fractal Flattening)" and "適応型マスク構築"): the
  * same outputs as nabla_flatten(q_grid -> q), nabla_flatten(k_grid -> k)
  * followed by nabla_build_mask(q, k), with the pooling done in the flattening
- * pass instead of re-reading the flattened copies.
+ * pass instead of re-reading the flattened copies, and the flattening of one
+ * head running beside the scores and cut of the previous one (one persistent
+ * launch; its device-side waits are bounded and report NABLA_ERR_TIMEOUT
+ * through nabla_status()).
  *   q_grid, k_grid  [B, heads, T, H, W, D] bf16 in grid order (inputs);
  *   q, k            [B, heads, N, D] bf16, written in flattened order (outputs;
  *                   the attention calls take them);

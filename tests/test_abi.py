@@ -51,7 +51,9 @@ def test_sizes(L):
     assert nabla.mask_bytes(s, nabla.MASK_BITS) == BH * nb * ((nb + 31) // 32) * 4
     assert nabla.mask_bytes(s, nabla.MASK_ROW_IDX) == BH * nb * nb * 2
     assert nabla.mask_bytes(s, nabla.MASK_COL_CNT) == BH * nb * 4
-    assert nabla.workspace_size(s, nabla.OP_BUILD_MASK) == 256 + 2 * BH * nb * D * 4
+    # status word, task counters of the persistent front end, pooled Q and K
+    ctr = (4 * (1 + BH) + 255) // 256 * 256
+    assert nabla.workspace_size(s, nabla.OP_BUILD_MASK) == 256 + ctr + 2 * BH * nb * D * 4
     assert nabla.workspace_size(s, nabla.OP_ATTN_BWD) == 256 + 2 * BH * N * 4
     assert nabla.workspace_size(s, nabla.OP_ATTN_FWD) >= 256
     # invalid shapes size to 0

@@ -53,6 +53,12 @@ def test_ragged_shapes(w):
         assert check_mask(to_np(c.gpu_mask(p)), c.oracle_mask(p)) == 0
 
 
+def _pooled_offset(w):
+    """Byte offset of the pooled Q in a mask workspace: after the 256-byte
+    status region and the front end's task counters (1 + B*heads ints)."""
+    return 256 + (4 * (1 + w.BH) + 255) // 256 * 256
+
+
 def test_pooled_means_bit_exact(small):
     w = small.w
     ws = nabla.workspace(small.shape, nabla.OP_BUILD_MASK, "cuda")
@@ -60,8 +66,9 @@ def test_pooled_means_bit_exact(small):
     torch.cuda.synchronize()
     n = w.BH * w.nb * w.D
     raw = ws.cpu().numpy()
-    qbar = raw[256:256 + 4 * n].view(np.float32).reshape(w.BH, w.nb, w.D)
-    off = 256 + ((4 * n + 255) // 256) * 256
+    base = _pooled_offset(w)
+    qbar = raw[base:base + 4 * n].view(np.float32).reshape(w.BH, w.nb, w.D)
+    off = base + ((4 * n + 255) // 256) * 256
     nbp = (w.nb + 3) // 4 * 4  # row stride of the transposed pooled K
     kbar_t = raw[off:off + 4 * w.BH * w.D * nbp].view(np.float32).reshape(w.BH, w.D, nbp)
     assert np.array_equal(qbar, oracle.pool_f32(small.cpu["q"]))
@@ -133,7 +140,8 @@ def test_build_mask_from_grid_matches_flatten_then_build(w, p, flags):
     if p is None:  # the scored path pooled from the grid layout
         n = w.BH * w.nb * w.D
         raw = ws.cpu().numpy()
-        qbar = raw[256:256 + 4 * n].view(np.float32).reshape(w.BH, w.nb, w.D)
+        base = _pooled_offset(w)
+        qbar = raw[base:base + 4 * n].view(np.float32).reshape(w.BH, w.nb, w.D)
         assert np.array_equal(qbar, oracle.pool_f32(c.cpu["q"]))
 
 
@@ -198,3 +206,22 @@ def test_tied_scores(w, patterns):
         om = c.oracle_mask(p)
         assert check_mask(gm, om) == 0
         _check_debug_scores(c, p)
+
+
+def test_front_end_wait_timeout_is_reported_and_the_context_survives():
+    # nabla_build_mask_grid runs the pooling and the scores in one persistent
+    # launch whose score tiles wait (bounded) for their head's pooling.  The
+    # test aid makes every such wait expect one tile too many with a 1 ms
+    # limit: the status must read NABLA_ERR_TIMEOUT, and the next call on the
+    # same context and workspace must be correct.
+    w = GRID[1]
+    c = Case(w)
+    inp = synth.make_inputs(w, 0, with_dout=False)
+    qg = inp["q"].reshape(w.BH, w.N, w.D).cuda()
+    kg = inp["k"].reshape(w.BH, w.N, w.D).cuda()
+    ws = nabla.workspace(c.shape, nabla.OP_BUILD_MASK, "cuda")
+    nabla.build_mask_grid(c.shape, c.params(flags=nabla.DEBUG_TIMEOUT), qg, kg, ws=ws)
+    assert nabla.status(ws) == nabla.ERR_TIMEOUT
+    _, _, gm = nabla.build_mask_grid(c.shape, c.params(), qg, kg, ws=ws)
+    assert nabla.status(ws) == nabla.OK
+    assert check_mask(to_np(gm), c.oracle_mask()) == 0
