@@ -43,13 +43,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the sources no longer match, the bench reports no traffic rather than a
 # stale figure.
 NCU_DRAM = {
-    # pre 317.0 + 3.7 MB, dK/dV 661.1 + 292.1 MB, dQ 646.4 + 141.9 MB at 8 heads
-    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.65e6 + 661.14e6 + 292.06e6
-                                               + 646.42e6 + 141.87e6) / 8,
-                            "sources_sha": "5a197c27ba01"},
-    # 475.2 + 145.5 MB at 8 heads
-    ("train", "attn_fwd"): {"bytes_per_head": (475.19e6 + 145.54e6) / 8,
-                            "sources_sha": "b3658f1cf267"},
+    # pre 317.0 + 3.8 MB, dK/dV 660.9 + 292.5 MB, dQ 650.7 + 142.8 MB at 8 heads
+    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.82e6 + 660.90e6 + 292.46e6
+                                               + 650.72e6 + 142.83e6) / 8,
+                            "sources_sha": "30c21cb13599"},
+    # 475.7 + 140.8 MB at 8 heads
+    ("train", "attn_fwd"): {"bytes_per_head": (475.67e6 + 140.76e6) / 8,
+                            "sources_sha": "73731400b2a3"},
 }
 KERNEL_SOURCES = {
     "attn_bwd": ("attn_bwd_sm100.cu", "sm100.cuh", "common.cuh"),
@@ -490,7 +490,9 @@ def run_nabla(args):
         for n in ("o", "dq", "dk", "dv"):
             nabla.flatten(B[n], w.T, w.H, w.W, w.P, inverse=True, out=out[n])
 
-    launches_per_step = 1 + 3 + 1 + 3 + 4  # flatten v, flatten_pool/score_cut/cols, fwd, bwd x3, unflatten
+    # flatten v; the persistent front end (flatten + pool of Q, K with scores and
+    # cut) and the column lists; fwd; pre, dK/dV, dQ; 4 unflattens
+    launches_per_step = 1 + 2 + 1 + 3 + 4
 
     def barrier():
         if world > 1:
