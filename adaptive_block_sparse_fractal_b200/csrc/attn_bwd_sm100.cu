@@ -214,20 +214,25 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         // MMA issuer: whole warp, one elected lane issues
         constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // K . Q^T, V . dO^T
         constexpr uint32_t kIdG = idesc_bf16(128, D, 0, 1);     // P^T . dO, dS^T . Q
+        // Shared-memory descriptors advance by (byte offset >> 4) in their low
+        // 14-bit address field; every tile address here stays below 2^18.
+        const uint64_t dK = desc_sw128(sb + KV_K, 16, 1024), dV = desc_sw128(sb + KV_V, 16, 1024);
         auto SdP = [&](int t) -> bool {
             const int s = t % kStages;
             if (!warp_wait(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
                 return false;
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
+            const uint64_t dQ = desc_sw128(st, 16, 1024), dO = desc_sw128(st + kQBytes, 16, 1024);
+            const uint32_t s0 = tmem + (t & 1) * 64, p0 = tmem + 128 + (t & 1) * 64;
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t ka = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                const uint32_t kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_ss_warp(tmem + (t & 1) * 64, desc_sw128(sb + KV_K + ka, 16, 1024),
-                            desc_sw128(st + kb, 16, 1024), kIdS, kk > 0);
-                mma_ss_warp(tmem + 128 + (t & 1) * 64, desc_sw128(sb + KV_V + ka, 16, 1024),
-                            desc_sw128(st + kQBytes + kb, 16, 1024), kIdS, kk > 0);
+            for (int kk = 0; kk < D / 16; kk += 2) {  // S^T, dP^T for k-steps kk and kk + 1
+                const uint32_t a0 = ((kk >> 2) * kHalfTile + (kk & 3) * 32) >> 4;
+                const uint32_t a1 = (((kk + 1) >> 2) * kHalfTile + ((kk + 1) & 3) * 32) >> 4;
+                const uint32_t b0 = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                const uint32_t b1 = (((kk + 1) >> 2) * 8192 + ((kk + 1) & 3) * 32) >> 4;
+                mma_ss4_warp(s0, p0, s0, p0, dK + a0, dV + a0, dK + a1, dV + a1, dQ + b0, dO + b0,
+                             dQ + b1, dO + b1, kIdS, kk > 0, kk > 0);
             }
             mma_commit_warp(&s_full[t & 1]);
             return true;
@@ -238,15 +243,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 return false;
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
-#pragma unroll
-            for (int kk = 0; kk < 64 / 16; ++kk) {  // queries 16kk.. at column 32(kk/2) + 8(kk%2)
-                const uint32_t acc = (t > 0 || kk > 0) ? 1u : 0u;
-                const uint32_t col = (t & 1) * 64 + 32 * (kk >> 1) + 8 * (kk & 1);
-                mma_ts_warp(tmem + 256, tmem + col, desc_sw128(st + kQBytes + kk * 2048, 8192, 1024),
-                            kIdG, acc);
-                mma_ts_warp(tmem + 384, tmem + 128 + col, desc_sw128(st + kk * 2048, 8192, 1024),
-                            kIdG, acc);
-            }
+            // dO, Q as MN-major B operands; query k-step kk (16 queries) starts
+            // 2048 bytes further and reads bf16 P^T / dS^T columns
+            // 32 (kk / 2) + 8 (kk % 2) of this tile's S^T / dP^T buffers
+            const uint64_t gO = desc_sw128(st + kQBytes, 8192, 1024), gQ = desc_sw128(st, 8192, 1024);
+            const uint32_t c = tmem + (t & 1) * 64;
+            const uint32_t f = t > 0 ? 1u : 0u;
+            mma_ts4_warp(tmem + 256, tmem + 384, tmem + 256, tmem + 384, c, c + 128, c + 8, c + 136,
+                         gO, gQ, gO + 128, gQ + 128, kIdG, f, f);
+            mma_ts4_warp(tmem + 256, tmem + 384, tmem + 256, tmem + 384, c + 32, c + 160, c + 40,
+                         c + 168, gO + 256, gQ + 256, gO + 384, gQ + 384, kIdG, 1u, 1u);
             mma_commit_warp(&st_empty[s]);
             return true;
         };
@@ -503,12 +509,15 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             tc_fence_after();
             const uint32_t b0 = sRing + slot * kDqSlot;
             const uint32_t d = tmem + (t & 1) * 128;
+            // descriptors advance by (byte offset >> 4) in their low address field
+            const uint64_t dK = desc_sw128(b0, 16, 1024), dV = desc_sw128(b0 + kBlockBytes, 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t off = (kk >> 2) * 8192 + (kk & 3) * 32;
-                mma_ts_warp(d, tmem + kColQ + 8 * kk, desc_sw128(b0 + off, 16, 1024), kIdS, kk > 0);
-                mma_ts_warp(d + 64, tmem + kColDO + 8 * kk,
-                            desc_sw128(b0 + kBlockBytes + off, 16, 1024), kIdS, kk > 0);
+            for (int kk = 0; kk < D / 16; kk += 2) {  // S, dP for k-steps kk and kk + 1
+                const uint32_t o0 = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                const uint32_t o1 = (((kk + 1) >> 2) * 8192 + ((kk + 1) & 3) * 32) >> 4;
+                mma_ts4_warp(d, d + 64, d, d + 64, tmem + kColQ + 8 * kk, tmem + kColDO + 8 * kk,
+                             tmem + kColQ + 8 * kk + 8, tmem + kColDO + 8 * kk + 8, dK + o0, dV + o0,
+                             dK + o1, dV + o1, kIdS, kk > 0, kk > 0);
             }
             mma_commit_warp(&s_full[t & 1]);
             return true;
@@ -518,11 +527,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             if (!warp_wait(&ds_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit))
                 return false;
             tc_fence_after();
-            const uint32_t b0 = sRing + slot * kDqSlot;
-#pragma unroll
-            for (int kk = 0; kk < 64 / 16; ++kk)  // keys 16kk.. at column 32(kk/2) + 8(kk%2)
-                mma_ts_warp(tmem + kColDQ, tmem + (t & 1) * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
-                       desc_sw128(b0 + kk * 2048, 8192, 1024), kIdQ, (t > 0 || kk > 0));
+            // K as the MN-major B operand: key k-step kk starts 2048 bytes further
+            // and reads bf16 dS columns 32 (kk / 2) + 8 (kk % 2) of this tile's S
+            const uint64_t gK = desc_sw128(sRing + slot * kDqSlot, 8192, 1024);
+            const uint32_t c = tmem + (t & 1) * 128;
+            mma_ts4_warp(tmem + kColDQ, tmem + kColDQ, tmem + kColDQ, tmem + kColDQ, c, c + 8, c + 32,
+                         c + 40, gK, gK + 128, gK + 256, gK + 384, kIdQ, t > 0 ? 1u : 0u, 1u);
             mma_commit_warp(&kv_empty[slot]);
             return true;
         };
@@ -640,7 +650,6 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 }  // namespace bwd100
 }  // namespace nabla
 
-bool nabla_make_tmap_rows(CUtensorMap *m, const void *base, uint64_t rows, int D);
 
 template <int D>
 static cudaError_t launch_bwd(int64_t BH, int nb, int Hp, int Wp, int T, float scale,

@@ -119,6 +119,41 @@ __device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, ui
         " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
+// Four MMAs behind one elect.sync (warp-collective like the above): MMA i is
+// D_i (+)= A_i * B_i.  MMAs 0 and 1 accumulate when acc0 / acc1 is nonzero,
+// MMAs 2 and 3 always accumulate.  The tensor core accepts an MMA roughly when
+// it starts executing it, so the issuing warp spends about an N = 64 MMA's
+// execution time per issue; fewer instructions per MMA keep the issue loop
+// from falling behind the pipe.
+__device__ __forceinline__ void mma_ss4_warp(uint32_t d0, uint32_t d1, uint32_t d2, uint32_t d3,
+                                             uint64_t a0, uint64_t a1, uint64_t a2, uint64_t a3,
+                                             uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3,
+                                             uint32_t idesc, uint32_t acc0, uint32_t acc1) {
+    asm volatile(
+        "{\n .reg .pred e, p0, p1, pt;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p0, %13, 0;\n"
+        " setp.ne.b32 p1, %14, 0;\n setp.ne.b32 pt, %12, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %12, p0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %5, %9, %12, p1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%2], %6, %10, %12, pt;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%3], %7, %11, %12, pt;\n}\n" ::"r"(d0),
+        "r"(d1), "r"(d2), "r"(d3), "l"(a0), "l"(a1), "l"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2),
+        "l"(b3), "r"(idesc), "r"(acc0), "r"(acc1));
+}
+// As mma_ss4_warp with the A operands in TMEM (column addresses a0..a3).
+__device__ __forceinline__ void mma_ts4_warp(uint32_t d0, uint32_t d1, uint32_t d2, uint32_t d3,
+                                             uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3,
+                                             uint32_t idesc, uint32_t acc0, uint32_t acc1) {
+    asm volatile(
+        "{\n .reg .pred e, p0, p1, pt;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p0, %13, 0;\n"
+        " setp.ne.b32 p1, %14, 0;\n setp.ne.b32 pt, %12, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %12, p0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%1], [%5], %9, %12, p1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%2], [%6], %10, %12, pt;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%3], [%7], %11, %12, pt;\n}\n" ::"r"(d0),
+        "r"(d1), "r"(d2), "r"(d3), "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2),
+        "l"(b3), "r"(idesc), "r"(acc0), "r"(acc1));
+}
 // Single-thread forms, for an issuer whose MMAs are N = 128 or wider (then
 // the issue cost is hidden behind execution and the warp's other lanes stay
 // out of the issuing path).
@@ -285,13 +320,16 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
         : "memory");
 }
 
-// wait_bar for a converged warp: lane 0 waits, the warp synchronises on it and
-// every lane returns lane 0's result.
+// wait_bar for a converged warp.  Every lane tests the barrier and the warp
+// votes, so no lane leaves the others: a completed phase costs ~30 cycles this
+// way, against ~180 for a test by lane 0 alone followed by a shuffle of its
+// answer.  Otherwise every lane runs the bounded wait and the warp returns
+// true only if all lanes saw the phase complete.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
                                           int *status, uint32_t limit_ns) {
-    int ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort, status, limit_ns) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    const bool ok = wait_bar(bar, parity, abort, status, limit_ns);
+    return __all_sync(0xffffffffu, ok);
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight work).
@@ -307,6 +345,6 @@ __device__ __forceinline__ bool wait_plain(uint64_t *bar, uint32_t parity, uint3
 }  // namespace sm100
 }  // namespace nabla
 
-// Host: TMA map over a [rows, 128] bf16 row-major tensor, boxes of 64 rows x
-// 64 features, 128-byte swizzle (defined in attn_fwd_sm100.cu).
-bool nabla_make_tmap_rows128(CUtensorMap *m, const void *base, uint64_t rows);
+// Host: TMA map over a [rows, D] bf16 row-major tensor (D = 64 or 128), boxes
+// of 64 rows x 64 features, 128-byte swizzle (defined in attn_fwd_sm100.cu).
+bool nabla_make_tmap_rows(CUtensorMap *m, const void *base, uint64_t rows, int D);
