@@ -43,13 +43,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the sources no longer match, the bench reports no traffic rather than a
 # stale figure.
 NCU_DRAM = {
-    # pre 317.0 + 3.8 MB, dK/dV 660.9 + 292.5 MB, dQ 650.7 + 142.8 MB at 8 heads
-    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.82e6 + 660.90e6 + 292.46e6
-                                               + 650.72e6 + 142.83e6) / 8,
-                            "sources_sha": "30c21cb13599"},
-    # 475.7 + 140.8 MB at 8 heads
-    ("train", "attn_fwd"): {"bytes_per_head": (475.67e6 + 140.76e6) / 8,
-                            "sources_sha": "73731400b2a3"},
+    # pre 317.0 + 4.0 MB, dK/dV 654.3 + 292.5 MB, dQ 649.8 + 143.1 MB at 8 heads
+    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 4.01e6 + 654.28e6 + 292.47e6
+                                               + 649.77e6 + 143.11e6) / 8,
+                            "sources_sha": "860ffbcc9f7f"},
+    # 477.6 + 140.3 MB at 8 heads
+    ("train", "attn_fwd"): {"bytes_per_head": (477.62e6 + 140.33e6) / 8,
+                            "sources_sha": "ef3835975990"},
 }
 KERNEL_SOURCES = {
     "attn_bwd": ("attn_bwd_sm100.cu", "sm100.cuh", "common.cuh"),
