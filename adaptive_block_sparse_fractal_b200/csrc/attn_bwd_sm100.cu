@@ -12,9 +12,12 @@
 // dkdv_kernel: one CTA per pair of temporally adjacent KEY blocks (128 key
 //   rows on the M = 128 datapath), walking the union of their mask columns,
 //   one query block (64 queries) per tile:
-//     S^T  = K . Q^T,  dP^T = V . dO^T                 (TMEM, double-buffered)
-//     P^T, dS^T = P^T (dP^T - D)  -> bf16 over S^T, dP^T in TMEM (two
-//                                    warpgroups, 32 queries each)
+//     S^T  = K . Q^T   (K resident in TMEM as the A operand; S^T double-
+//                       buffered)
+//     dP^T = V . dO^T  (V from shared memory; one dP^T buffer, refilled once
+//                       the softmax warps have loaded the previous tile's)
+//     P^T, dS^T = P^T (dP^T - D)  -> bf16, both over the tile's S^T columns
+//                                    (two warpgroups, 32 queries each)
 //     dV  += P^T . dO,  dK += dS^T . Q                  (TMEM A operands and
 //                                                        accumulators)
 // dq_kernel: one CTA per pair of temporally adjacent QUERY blocks (128 query
@@ -72,31 +75,35 @@ __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restric
 // ---------------------------------------------------------------------------
 constexpr int kStages = 3;
 constexpr int kKvThreads = 320;
-// shared memory of the dK/dV kernel for head dim D: K and V of the key pair
+// shared memory of the dK/dV kernel for head dim D: V of the key pair
 // (resident), then a ring of query stages (Q, dO, -L log2 e, -D)
 template <int D>
 struct KvLayout {
     static constexpr int kHalves = D / 64;
     static constexpr uint32_t kQBytes = 64u * D * 2;                   // one query block
     static constexpr uint32_t kStageBytes = ((2 * kQBytes + 512 + 1023) / 1024) * 1024;
-    static constexpr uint32_t KV_K = 0, KV_V = kHalves * kHalfTile;
-    static constexpr uint32_t KV_RING = 2 * kHalves * kHalfTile;
+    static constexpr uint32_t KV_V = 0;
+    static constexpr uint32_t KV_RING = kHalves * kHalfTile;
     static constexpr uint32_t KV_U = KV_RING + kStages * kStageBytes;  // union list
     static constexpr uint32_t KV_UF = KV_U + 2 * (kMaxNbBwd + 8);
     static constexpr uint32_t KV_CB = ((KV_UF + kMaxNbBwd + 8 + 15) / 16) * 16;  // col bits [2][64]
     static constexpr uint32_t KV_BAR = KV_CB + 2 * 256;
-    static constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1;
+    static constexpr int kKvBars = 1 + 2 * kStages + 2 + 2 + 1 + 1 + 2;
     static constexpr uint32_t KV_INT = KV_BAR + 8 * kKvBars;
     static constexpr uint32_t kKvSmem = KV_INT + 16 + 1024;
 };
 
-// TMEM columns: S^T(t) [64 (t&1), +64), dP^T(t) [128 + 64 (t&1), +64),
+// TMEM columns: S^T(t) [64 (t&1), +64), dP^T [128, 192), K [192, 192 + D/2),
 // dV [256, 256 + D), dK [384, 384 + D).  Warpgroup qg handles queries
-// [32 qg, +32) of the tile and writes bf16 P^T and dS^T for them over the
-// first 16 of its own S^T and dP^T columns, where the dV and dK MMAs read them.
+// [32 qg, +32) of the tile and writes bf16 P^T and dS^T for them over its own
+// S^T columns, P^T at [32 qg, +16) and dS^T at [32 qg + 16, +16), where the dV
+// and dK MMAs read them.  With K as a TMEM operand, S^T reads only Q from
+// shared memory: the shared-memory operands of both N = 64 MMAs (6 KB each)
+// were above what the tensor core draws from shared memory per cycle.
+constexpr uint32_t kColDP = 128, kColK = 192;
 template <int D>
 __global__ void __launch_bounds__(kKvThreads, 1)
-    dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+    dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __nv_bfloat16 *__restrict__ k,
                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                 const float *__restrict__ l2, const float *__restrict__ dl,
                 const uint16_t *__restrict__ col_idx, const int32_t *__restrict__ col_cnt,
@@ -106,7 +113,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     using L = KvLayout<D>;
     constexpr int kHalves = L::kHalves;
     constexpr uint32_t kQBytes = L::kQBytes, kStageBytes = L::kStageBytes;
-    constexpr uint32_t KV_K = L::KV_K, KV_V = L::KV_V, KV_RING = L::KV_RING, KV_U = L::KV_U,
+    constexpr uint32_t KV_V = L::KV_V, KV_RING = L::KV_RING, KV_U = L::KV_U,
                        KV_UF = L::KV_UF, KV_CB = L::KV_CB, KV_BAR = L::KV_BAR, KV_INT = L::KV_INT;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -122,6 +129,9 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     // barriers, so a warp already on tile t+1 cannot complete tile t's phase)
     uint64_t *s_full = bar + 1 + 2 * kStages, *pd_full = s_full + 2, *done = pd_full + 2;
     uint64_t *never = done + 1;  // nothing arrives here (timeout test aid)
+    // k_ready: the eight softmax warps stored K in TMEM; dp_free: they loaded
+    // the dP^T of their current tile (the buffer may be refilled)
+    uint64_t *k_ready = never + 1, *dp_free = k_ready + 1;
     int *sInt = reinterpret_cast<int *>(sm + KV_INT);
     volatile int *abort_flag = sInt + 2;
 
@@ -148,6 +158,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         }
         mbar_init(done, 1);
         mbar_init(never, 1);
+        mbar_init(k_ready, 8);
+        mbar_init(dp_free, 8);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
     }
@@ -181,14 +193,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tq);
-        prefetch_tmap(&tk);
         prefetch_tmap(&tv);
         prefetch_tmap(&tdo);
         const int ya = row_base + jA * kBlk, yb = row_base + (jB >= 0 ? jB : jA) * kBlk;
-        mbar_expect_tx(kv_full, 2 * kHalves * kHalfTile);
+        mbar_expect_tx(kv_full, kHalves * kHalfTile);
         for (int dh = 0; dh < kHalves; ++dh) {
-            tma_load_2d(sb + KV_K + dh * kHalfTile, &tk, kv_full, 64 * dh, ya);
-            tma_load_2d(sb + KV_K + dh * kHalfTile + 8192, &tk, kv_full, 64 * dh, yb);
             tma_load_2d(sb + KV_V + dh * kHalfTile, &tv, kv_full, 64 * dh, ya);
             tma_load_2d(sb + KV_V + dh * kHalfTile + 8192, &tv, kv_full, 64 * dh, yb);
         }
@@ -216,23 +225,26 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         constexpr uint32_t kIdG = idesc_bf16(128, D, 0, 1);     // P^T . dO, dS^T . Q
         // Shared-memory descriptors advance by (byte offset >> 4) in their low
         // 14-bit address field; every tile address here stays below 2^18.
-        const uint64_t dK = desc_sw128(sb + KV_K, 16, 1024), dV = desc_sw128(sb + KV_V, 16, 1024);
+        const uint64_t dV = desc_sw128(sb + KV_V, 16, 1024);
         auto SdP = [&](int t) -> bool {
             const int s = t % kStages;
             if (!warp_wait(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
                 return false;
+            // the single dP^T buffer: the softmax warps hold tile t - 1's in registers
+            if (t > 0 && !warp_wait(dp_free, (t - 1) & 1, abort_flag, status, wait_limit))
+                return false;
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
             const uint64_t dQ = desc_sw128(st, 16, 1024), dO = desc_sw128(st + kQBytes, 16, 1024);
-            const uint32_t s0 = tmem + (t & 1) * 64, p0 = tmem + 128 + (t & 1) * 64;
+            const uint32_t s0 = tmem + (t & 1) * 64, p0 = tmem + kColDP;
 #pragma unroll
             for (int kk = 0; kk < D / 16; kk += 2) {  // S^T, dP^T for k-steps kk and kk + 1
                 const uint32_t a0 = ((kk >> 2) * kHalfTile + (kk & 3) * 32) >> 4;
                 const uint32_t a1 = (((kk + 1) >> 2) * kHalfTile + ((kk + 1) & 3) * 32) >> 4;
                 const uint32_t b0 = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
                 const uint32_t b1 = (((kk + 1) >> 2) * 8192 + ((kk + 1) & 3) * 32) >> 4;
-                mma_ss4_warp(s0, p0, s0, p0, dK + a0, dV + a0, dK + a1, dV + a1, dQ + b0, dO + b0,
-                             dQ + b1, dO + b1, kIdS, kk > 0, kk > 0);
+                mma_tsss4_warp(s0, p0, s0, p0, tmem + kColK + 8 * kk, dV + a0, tmem + kColK + 8 * kk + 8,
+                               dV + a1, dQ + b0, dO + b0, dQ + b1, dO + b1, kIdS, kk > 0, kk > 0);
             }
             mma_commit_warp(&s_full[t & 1]);
             return true;
@@ -245,18 +257,19 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const uint32_t st = sb + KV_RING + s * kStageBytes;
             // dO, Q as MN-major B operands; query k-step kk (16 queries) starts
             // 2048 bytes further and reads bf16 P^T / dS^T columns
-            // 32 (kk / 2) + 8 (kk % 2) of this tile's S^T / dP^T buffers
+            // 32 (kk / 2) + 8 (kk % 2) / + 16 of this tile's S^T buffer
             const uint64_t gO = desc_sw128(st + kQBytes, 8192, 1024), gQ = desc_sw128(st, 8192, 1024);
             const uint32_t c = tmem + (t & 1) * 64;
             const uint32_t f = t > 0 ? 1u : 0u;
-            mma_ts4_warp(tmem + 256, tmem + 384, tmem + 256, tmem + 384, c, c + 128, c + 8, c + 136,
+            mma_ts4_warp(tmem + 256, tmem + 384, tmem + 256, tmem + 384, c, c + 16, c + 8, c + 24,
                          gO, gQ, gO + 128, gQ + 128, kIdG, f, f);
-            mma_ts4_warp(tmem + 256, tmem + 384, tmem + 256, tmem + 384, c + 32, c + 160, c + 40,
-                         c + 168, gO + 256, gQ + 256, gO + 384, gQ + 384, kIdG, 1u, 1u);
+            mma_ts4_warp(tmem + 256, tmem + 384, tmem + 256, tmem + 384, c + 32, c + 48, c + 40,
+                         c + 56, gO + 256, gQ + 256, gO + 384, gQ + 384, kIdG, 1u, 1u);
             mma_commit_warp(&st_empty[s]);
             return true;
         };
-        if (ntiles > 0 && warp_wait(kv_full, 0, abort_flag, status, wait_limit)) {
+        if (ntiles > 0 && warp_wait(kv_full, 0, abort_flag, status, wait_limit) &&
+            warp_wait(k_ready, 0, abort_flag, status, wait_limit)) {
             bool ok = SdP(0);
             for (int t = 0; ok && t < ntiles; ++t) {
                 if (t + 1 < ntiles) ok = SdP(t + 1);
@@ -274,6 +287,32 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
         bool ok = true;
         if (force_timeout) ok = wait_bar(never, 0, abort_flag, status, 16);  // nothing arrives
+        {
+            // features [D/2 qg, D/2 qg + D/2) of key row tw -> TMEM columns
+            // [kColK + D/4 qg, +D/4): K as the A operand of S^T = K Q^T (a
+            // missing second block of the pair repeats the first; its rows are
+            // never written out)
+            const int jk = (kh && jB >= 0) ? jB : jA;
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                k + (static_cast<int64_t>(row_base) + jk * kBlk + (tw & 63)) * D + (D / 2) * qg);
+            uint32_t kv[D / 4];
+#pragma unroll
+            for (int e = 0; e < D / 16; ++e) {
+                const uint4 v = __ldg(src + e);
+                kv[4 * e] = v.x;
+                kv[4 * e + 1] = v.y;
+                kv[4 * e + 2] = v.z;
+                kv[4 * e + 3] = v.w;
+            }
+            if constexpr (D == 128)
+                tmem_st32(tmem + lane_base + kColK + 32 * qg, reinterpret_cast<float *>(kv));
+            else
+                tmem_st16(tmem + lane_base + kColK + 16 * qg, kv);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(k_ready);
         for (int t = 0; t < ntiles; ++t) {
             ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
@@ -286,8 +325,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 const float4 *D4 = L4 + 16;  // D follows L2 at +256 bytes
                 float sv[32], dp[32];
                 tmem_ld32(scol, sv);
-                tmem_ld32(scol + 128, dp);
+                tmem_ld32(tmem + lane_base + kColDP + 32 * qg, dp);
                 tmem_wait_ld();
+                // dP^T is in registers: the buffer may take the next tile's
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dp_free);
 #pragma unroll
                 for (int q4 = 0; q4 < 8; ++q4) {
                     const float4 l4 = L4[q4], d4 = D4[q4];
@@ -308,11 +351,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     }
                 }
             } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dp_free);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) pk[e] = dk2[e] = 0u;
             }
             tmem_st16(scol, pk);
-            tmem_st16(scol + 128, dk2);
+            tmem_st16(scol + 16, dk2);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -678,7 +724,8 @@ static cudaError_t launch_bwd(int64_t BH, int nb, int Hp, int Wp, int T, float s
     if (err != cudaSuccess) return err;
     const int64_t groups = static_cast<int64_t>((T + 1) / 2) * Hp * Wp;
     dkdv_kernel<D><<<static_cast<unsigned>(BH * groups), kKvThreads, kKvSmem, stream>>>(
-        mq, mk, mv, mdo, l2, dl, col_idx, col_cnt, static_cast<__nv_bfloat16 *>(dk),
+        mq, static_cast<const __nv_bfloat16 *>(k), mv, mdo, l2, dl, col_idx, col_cnt,
+        static_cast<__nv_bfloat16 *>(dk),
         static_cast<__nv_bfloat16 *>(dv), status, nb, Hp, Wp, T, c, scale, limit, force_timeout);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;

@@ -154,6 +154,22 @@ __device__ __forceinline__ void mma_ts4_warp(uint32_t d0, uint32_t d1, uint32_t 
         "r"(d1), "r"(d2), "r"(d3), "r"(a0), "r"(a1), "r"(a2), "r"(a3), "l"(b0), "l"(b1), "l"(b2),
         "l"(b3), "r"(idesc), "r"(acc0), "r"(acc1));
 }
+// As mma_ss4_warp with MMAs 0 and 2 taking their A operand from TMEM (a0, a2
+// column addresses) and MMAs 1 and 3 from shared memory (a1, a3 descriptors).
+__device__ __forceinline__ void mma_tsss4_warp(uint32_t d0, uint32_t d1, uint32_t d2, uint32_t d3,
+                                               uint32_t a0, uint64_t a1, uint32_t a2, uint64_t a3,
+                                               uint64_t b0, uint64_t b1, uint64_t b2, uint64_t b3,
+                                               uint32_t idesc, uint32_t acc0, uint32_t acc1) {
+    asm volatile(
+        "{\n .reg .pred e, p0, p1, pt;\n elect.sync _|e, 0xffffffff;\n setp.ne.b32 p0, %13, 0;\n"
+        " setp.ne.b32 p1, %14, 0;\n setp.ne.b32 pt, %12, 0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %12, p0;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%1], %5, %9, %12, p1;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%2], [%6], %10, %12, pt;\n"
+        " @e tcgen05.mma.cta_group::1.kind::f16 [%3], %7, %11, %12, pt;\n}\n" ::"r"(d0),
+        "r"(d1), "r"(d2), "r"(d3), "r"(a0), "l"(a1), "r"(a2), "l"(a3), "l"(b0), "l"(b1), "l"(b2),
+        "l"(b3), "r"(idesc), "r"(acc0), "r"(acc1));
+}
 // Single-thread forms, for an issuer whose MMAs are N = 128 or wider (then
 // the issue cost is hidden behind execution and the warp's other lanes stay
 // out of the issuing path).
