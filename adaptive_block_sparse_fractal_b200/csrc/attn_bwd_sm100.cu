@@ -73,7 +73,7 @@ __global__ void __launch_bounds__(256) pre_kernel(const __nv_bfloat16 *__restric
 // ---------------------------------------------------------------------------
 // dK, dV
 // ---------------------------------------------------------------------------
-constexpr int kStages = 3;
+constexpr int kStages = 4;
 constexpr int kKvThreads = 320;
 // shared memory of the dK/dV kernel for head dim D: V of the key pair
 // (resident), then a ring of query stages (Q, dO, -L log2 e, -D)
@@ -230,22 +230,34 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const int s = t % kStages;
             if (!warp_wait(&st_full[s], (t / kStages) & 1, abort_flag, status, wait_limit))
                 return false;
-            // the single dP^T buffer: the softmax warps hold tile t - 1's in registers
-            if (t > 0 && !warp_wait(dp_free, (t - 1) & 1, abort_flag, status, wait_limit))
-                return false;
             tc_fence_after();
             const uint32_t st = sb + KV_RING + s * kStageBytes;
             const uint64_t dQ = desc_sw128(st, 16, 1024), dO = desc_sw128(st + kQBytes, 16, 1024);
             const uint32_t s0 = tmem + (t & 1) * 64, p0 = tmem + kColDP;
+            // byte offsets of k-step kk (16 features) in a K-major tile of one
+            // key / query block pair: 64-feature halves kHalfTile / 8192 apart
+            auto offA = [](int kk) {
+                return static_cast<uint32_t>(((kk >> 2) * kHalfTile + (kk & 3) * 32) >> 4);
+            };
+            auto offB = [](int kk) {
+                return static_cast<uint32_t>(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
+            };
+            // S^T first (K from TMEM, Q from shared memory) ...
 #pragma unroll
-            for (int kk = 0; kk < D / 16; kk += 2) {  // S^T, dP^T for k-steps kk and kk + 1
-                const uint32_t a0 = ((kk >> 2) * kHalfTile + (kk & 3) * 32) >> 4;
-                const uint32_t a1 = (((kk + 1) >> 2) * kHalfTile + ((kk + 1) & 3) * 32) >> 4;
-                const uint32_t b0 = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                const uint32_t b1 = (((kk + 1) >> 2) * 8192 + ((kk + 1) & 3) * 32) >> 4;
-                mma_tsss4_warp(s0, p0, s0, p0, tmem + kColK + 8 * kk, dV + a0, tmem + kColK + 8 * kk + 8,
-                               dV + a1, dQ + b0, dO + b0, dQ + b1, dO + b1, kIdS, kk > 0, kk > 0);
-            }
+            for (int kk = 0; kk < D / 16; kk += 4)
+                mma_ts4_warp(s0, s0, s0, s0, tmem + kColK + 8 * kk, tmem + kColK + 8 * kk + 8,
+                             tmem + kColK + 8 * kk + 16, tmem + kColK + 8 * kk + 24, dQ + offB(kk),
+                             dQ + offB(kk + 1), dQ + offB(kk + 2), dQ + offB(kk + 3), kIdS, kk > 0, 1u);
+            // ... then dP^T into the single buffer, once the softmax warps hold
+            // tile t - 1's in registers
+            if (t > 0 && !warp_wait(dp_free, (t - 1) & 1, abort_flag, status, wait_limit))
+                return false;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk += 4)
+                mma_ss4_warp(p0, p0, p0, p0, dV + offA(kk), dV + offA(kk + 1), dV + offA(kk + 2),
+                             dV + offA(kk + 3), dO + offB(kk), dO + offB(kk + 1), dO + offB(kk + 2),
+                             dO + offB(kk + 3), kIdS, kk > 0, 1u);
             mma_commit_warp(&s_full[t & 1]);
             return true;
         };
