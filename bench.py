@@ -43,13 +43,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the sources no longer match, the bench reports no traffic rather than a
 # stale figure.
 NCU_DRAM = {
-    # pre 317.0 + 4.0 MB, dK/dV 654.3 + 292.5 MB, dQ 649.8 + 143.1 MB at 8 heads
-    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 4.01e6 + 654.28e6 + 292.47e6
-                                               + 649.77e6 + 143.11e6) / 8,
-                            "sources_sha": "860ffbcc9f7f"},
-    # 477.6 + 140.3 MB at 8 heads
-    ("train", "attn_fwd"): {"bytes_per_head": (477.62e6 + 140.33e6) / 8,
-                            "sources_sha": "ef3835975990"},
+    # pre 317.0 + 3.8 MB, dK/dV 655.4 + 293.1 MB, dQ 649.1 + 143.4 MB at 8 heads
+    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.82e6 + 655.42e6 + 293.13e6
+                                               + 649.06e6 + 143.35e6) / 8,
+                            "sources_sha": "0054744bff9d"},
+    # 476.3 + 140.6 MB at 8 heads
+    ("train", "attn_fwd"): {"bytes_per_head": (476.34e6 + 140.63e6) / 8,
+                            "sources_sha": "9ea9d3d0ece4"},
 }
 KERNEL_SOURCES = {
     "attn_bwd": ("attn_bwd_sm100.cu", "sm100.cuh", "common.cuh"),
