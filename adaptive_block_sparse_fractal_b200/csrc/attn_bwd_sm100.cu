@@ -422,8 +422,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // One CTA per pair of temporally adjacent QUERY blocks (128 query rows on the
 // M = 128 datapath, the same pairing as the forward), walking the union of
 // their mask rows one key block (64 keys) per tile:
-//   S  = Q . K^T,  dP = dO . V^T    (Q, dO are TMEM A operands; S, dP double-
-//                                    buffered in TMEM)
+//   S  = Q . K^T,  dP = dO . V^T    (Q, dO are TMEM A operands; S in three
+//                                    TMEM buffers, dP in one)
 //   dS = P (dP - D)  -> bf16, written over S in TMEM
 //   dQ += dS . K                     (dS the TMEM A operand, K from shared
 //                                    memory, MN-major; accumulator in TMEM)
@@ -431,10 +431,16 @@ __global__ void __launch_bounds__(kKvThreads, 1)
 // (g, r) handles query row r and keys [32 g, 32 g + 32) of the tile, and
 // writes their bf16 dS over its own S columns [32 g, 32 g + 16).
 // Queries of the pair whose own row does not keep a key block get dS = 0.
-// TMEM columns: buffer b in [128 b, 128 b + 128) holds S (64) then dP (64);
-// dQ [256, 256 + D), Q [384, 384 + D/2), dO [448, 448 + D/2).
-constexpr int kDqThreads = 320;
-constexpr uint32_t kColDQ = 256, kColQ = 384, kColDO = 448;
+// Two warps issue the MMAs: warp 1 the S and dP MMAs, warp 10 the dQ MMAs.
+// With three S buffers the S MMAs of tile t only wait for the dQ MMAs of
+// tile t - 3, and the one dP buffer is refilled once the dS warps have loaded
+// tile t - 1's dP into registers, so neither issuer waits on the other's
+// latest work and the tensor pipe takes whichever stream is ready.
+// TMEM columns: S(t) [64 (t % 3), +64), dP [192, 256), dQ [256, 256 + D),
+// Q [384, 384 + D/2), dO [448, 448 + D/2).
+constexpr int kDqThreads = 352;
+constexpr int kDqGradWarp = 10;
+constexpr uint32_t kDqColDP = 192, kColDQ = 256, kColQ = 384, kColDO = 448;
 template <int D>
 struct DqLayout {
     static constexpr int kHalves = D / 64;
@@ -446,7 +452,7 @@ struct DqLayout {
     static constexpr uint32_t DQ_U = DQ_RB + 2 * 256;                // union list u16
     static constexpr uint32_t DQ_UF = DQ_U + 2 * (kMaxNbBwd + 8);    // membership per entry
     static constexpr uint32_t DQ_BAR = ((DQ_UF + kMaxNbBwd + 8 + 7) / 8) * 8;
-    static constexpr int kDqBars = 2 * kDqRing + 2 + 2 + 1 + 1 + 1;
+    static constexpr int kDqBars = 2 * kDqRing + 3 + 3 + 1 + 1 + 1 + 3 + 1 + 1;
     static constexpr uint32_t DQ_INT = DQ_BAR + 8 * kDqBars;
     static constexpr uint32_t kDqSmem = DQ_INT + 16 + 1024;
 };
@@ -474,10 +480,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     uint8_t *uFlag = sm + DQ_UF;
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + DQ_BAR);
     uint64_t *kv_full = bar, *kv_empty = bar + kDqRing, *s_full = bar + 2 * kDqRing;
-    // ds_full[t & 1]: the eight dS warps wrote dS(t) (two barriers, so a warp
-    // already on tile t+1 cannot complete tile t's phase for the others)
-    uint64_t *ds_full = s_full + 2, *q_ready = ds_full + 2, *done = q_ready + 1;
+    // per S buffer t % 3: s_full (S(t), dP(t) complete), ds_full (the eight dS
+    // warps wrote dS(t)), s_free (the dQ MMAs of tile t read it)
+    uint64_t *ds_full = s_full + 3, *q_ready = ds_full + 3, *done = q_ready + 1;
     uint64_t *never = done + 1;  // nothing arrives here (timeout test aid)
+    uint64_t *s_free = never + 1;
+    // dp_free: the dS warps loaded the current tile's dP (the buffer may be
+    // refilled); sdp_done: every S / dP MMA finished
+    uint64_t *dp_free = s_free + 3, *sdp_done = dp_free + 1;
     int *sInt = reinterpret_cast<int *>(sm + DQ_INT);  // [0] tmem base [1] tiles [2] abort
     volatile int *abort_flag = sInt + 2;
 
@@ -497,13 +507,16 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             mbar_init(&kv_full[r], 1);
             mbar_init(&kv_empty[r], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < 3; ++b) {
             mbar_init(&s_full[b], 1);
             mbar_init(&ds_full[b], 8);
+            mbar_init(&s_free[b], 1);
         }
         mbar_init(q_ready, 8);
         mbar_init(done, 1);
         mbar_init(never, 1);
+        mbar_init(dp_free, 8);
+        mbar_init(sdp_done, 1);
         sInt[2] = *reinterpret_cast<volatile int *>(status) != 0 ? 1 : 0;
         fence_mbar_init();
     }
@@ -557,49 +570,58 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         for (int u = t > kDqRing ? t - kDqRing : 0; u < t; ++u)
             wait_plain(&kv_full[u % kDqRing], (u / kDqRing) & 1, wait_limit);
     } else if (warp == 1) {
-        // ---------------- MMA issuer (whole warp, one elected lane issues) ----------------
+        // ---------------- S / dP issuer (whole warp, one elected lane issues) ----------------
         constexpr uint32_t kIdS = idesc_bf16(128, 64, 0, 0);    // Q . K^T, dO . V^T
-        constexpr uint32_t kIdQ = idesc_bf16(128, D, 0, 1);     // dS . K (K MN-major)
-        auto SdP = [&](int t) -> bool {
-            const int slot = t % kDqRing;
-            if (!warp_wait(&kv_full[slot], (t / kDqRing) & 1, abort_flag, status, wait_limit))
-                return false;
+        auto off = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 8192 + (kk & 3) * 32) >> 4); };
+        bool ok = ntiles > 0 && warp_wait(q_ready, 0, abort_flag, status, wait_limit);
+        for (int t = 0; ok && t < ntiles; ++t) {
+            const int slot = t % kDqRing, b = t % 3;
+            ok = warp_wait(&kv_full[slot], (t / kDqRing) & 1, abort_flag, status, wait_limit);
+            // S buffer t % 3 is free once the dQ MMAs of tile t - 3 have read its dS
+            if (ok && t >= 3)
+                ok = warp_wait(&s_free[b], ((t / 3) - 1) & 1, abort_flag, status, wait_limit);
+            if (!ok) break;
             tc_fence_after();
             const uint32_t b0 = sRing + slot * kDqSlot;
-            const uint32_t d = tmem + (t & 1) * 128;
+            const uint32_t d = tmem + 64 * b;
             // descriptors advance by (byte offset >> 4) in their low address field
             const uint64_t dK = desc_sw128(b0, 16, 1024), dV = desc_sw128(b0 + kBlockBytes, 16, 1024);
+            // S first ...
 #pragma unroll
-            for (int kk = 0; kk < D / 16; kk += 2) {  // S, dP for k-steps kk and kk + 1
-                const uint32_t o0 = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                const uint32_t o1 = (((kk + 1) >> 2) * 8192 + ((kk + 1) & 3) * 32) >> 4;
-                mma_ts4_warp(d, d + 64, d, d + 64, tmem + kColQ + 8 * kk, tmem + kColDO + 8 * kk,
-                             tmem + kColQ + 8 * kk + 8, tmem + kColDO + 8 * kk + 8, dK + o0, dV + o0,
-                             dK + o1, dV + o1, kIdS, kk > 0, kk > 0);
-            }
-            mma_commit_warp(&s_full[t & 1]);
-            return true;
-        };
-        auto Grad = [&](int t) -> bool {
-            const int slot = t % kDqRing;
-            if (!warp_wait(&ds_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit))
-                return false;
+            for (int kk = 0; kk < D / 16; kk += 4)
+                mma_ts4_warp(d, d, d, d, tmem + kColQ + 8 * kk, tmem + kColQ + 8 * kk + 8,
+                             tmem + kColQ + 8 * kk + 16, tmem + kColQ + 8 * kk + 24, dK + off(kk),
+                             dK + off(kk + 1), dK + off(kk + 2), dK + off(kk + 3), kIdS, kk > 0, 1u);
+            // ... then dP into the single buffer, once the dS warps hold tile
+            // t - 1's in registers
+            if (t > 0 && !warp_wait(dp_free, (t - 1) & 1, abort_flag, status, wait_limit)) break;
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < D / 16; kk += 4)
+                mma_ts4_warp(tmem + kDqColDP, tmem + kDqColDP, tmem + kDqColDP, tmem + kDqColDP,
+                             tmem + kColDO + 8 * kk, tmem + kColDO + 8 * kk + 8, tmem + kColDO + 8 * kk + 16,
+                             tmem + kColDO + 8 * kk + 24, dV + off(kk), dV + off(kk + 1), dV + off(kk + 2),
+                             dV + off(kk + 3), kIdS, kk > 0, 1u);
+            mma_commit_warp(&s_full[b]);
+        }
+        mma_commit_warp(sdp_done);  // completes once every MMA issued above has finished
+        if (lane == 0) wait_plain(sdp_done, 0, wait_limit);
+        __syncwarp();
+    } else if (warp == kDqGradWarp) {
+        // ---------------- dQ issuer (whole warp, one elected lane issues) ----------------
+        constexpr uint32_t kIdQ = idesc_bf16(128, D, 0, 1);     // dS . K (K MN-major)
+        for (int t = 0; t < ntiles; ++t) {
+            const int slot = t % kDqRing, b = t % 3;
+            if (!warp_wait(&ds_full[b], (t / 3) & 1, abort_flag, status, wait_limit)) break;
             tc_fence_after();
             // K as the MN-major B operand: key k-step kk starts 2048 bytes further
             // and reads bf16 dS columns 32 (kk / 2) + 8 (kk % 2) of this tile's S
             const uint64_t gK = desc_sw128(sRing + slot * kDqSlot, 8192, 1024);
-            const uint32_t c = tmem + (t & 1) * 128;
+            const uint32_t c = tmem + 64 * b;
             mma_ts4_warp(tmem + kColDQ, tmem + kColDQ, tmem + kColDQ, tmem + kColDQ, c, c + 8, c + 32,
                          c + 40, gK, gK + 128, gK + 256, gK + 384, kIdQ, t > 0 ? 1u : 0u, 1u);
             mma_commit_warp(&kv_empty[slot]);
-            return true;
-        };
-        if (ntiles > 0 && warp_wait(q_ready, 0, abort_flag, status, wait_limit)) {
-            bool ok = SdP(0);
-            for (int t = 0; ok && t < ntiles; ++t) {
-                if (t + 1 < ntiles) ok = SdP(t + 1);
-                ok = ok && Grad(t);
-            }
+            mma_commit_warp(&s_free[b]);
         }
         mma_commit_warp(done);  // completes once every MMA issued above has finished
         if (lane == 0) wait_plain(done, 0, wait_limit);
@@ -640,16 +662,20 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         if (lane == 0) mbar_arrive(q_ready);
 
         for (int t = 0; t < ntiles; ++t) {
-            ok = wait_bar(&s_full[t & 1], (t >> 1) & 1, abort_flag, status, wait_limit) && ok;
+            ok = wait_bar(&s_full[t % 3], (t / 3) & 1, abort_flag, status, wait_limit) && ok;
             tc_fence_after();
             const bool valid = (uFlag[t] >> h) & 1u;  // uniform per warp
-            const uint32_t scol = tmem + lane_base + (t & 1) * 128 + 32 * kg;
+            const uint32_t scol = tmem + lane_base + (t % 3) * 64 + 32 * kg;
             uint32_t gk[16];
             if (valid) {
                 float sv[32], dp[32];
                 tmem_ld32(scol, sv);
-                tmem_ld32(scol + 64, dp);
+                tmem_ld32(tmem + lane_base + kDqColDP + 32 * kg, dp);
                 tmem_wait_ld();
+                // dP is in registers: the buffer may take the next tile's
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dp_free);
                 const uint64_t c2 = f2_pack(c, c), nl2 = f2_pack(nLr, nLr), nd2 = f2_pack(nDr, nDr);
 #pragma unroll
                 for (int e = 0; e < 32; e += 2) {
@@ -659,6 +685,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     gk[e >> 1] = pack_bf16(f2_lo(g), f2_hi(g));
                 }
             } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dp_free);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) gk[e] = 0u;
             }
@@ -667,7 +696,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ds_full[t & 1]);
+            if (lane == 0) mbar_arrive(&ds_full[t % 3]);
         }
         // ---------------- epilogue: group kg writes dQ features [D/2 kg, D/2 kg + D/2) ----------------
         if (ok && ntiles > 0) ok = wait_bar(done, 0, abort_flag, status, wait_limit);
