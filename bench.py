@@ -43,12 +43,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the sources no longer match, the bench reports no traffic rather than a
 # stale figure.
 NCU_DRAM = {
-    # pre 317.0 + 3.8 MB, dK/dV 655.4 + 293.1 MB, dQ 649.1 + 143.4 MB at 8 heads
-    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.82e6 + 655.42e6 + 293.13e6
-                                               + 649.06e6 + 143.35e6) / 8,
-                            "sources_sha": "0054744bff9d"},
-    # 476.3 + 140.6 MB at 8 heads
-    ("train", "attn_fwd"): {"bytes_per_head": (476.34e6 + 140.63e6) / 8,
+    # pre 317.0 + 4.0 MB, dK/dV 653.4 + 292.6 MB, dQ 649.9 + 142.5 MB at 8 heads
+    ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.97e6 + 653.38e6 + 292.59e6
+                                               + 649.92e6 + 142.47e6) / 8,
+                            "sources_sha": "c4ee656f4caa"},
+    # 475.7 + 140.4 MB at 8 heads
+    ("train", "attn_fwd"): {"bytes_per_head": (475.69e6 + 140.43e6) / 8,
                             "sources_sha": "9ea9d3d0ece4"},
 }
 KERNEL_SOURCES = {
