@@ -568,10 +568,12 @@ def run_nabla(args):
         roofline["peak_at_clock"] = clk_peak
 
     # ---- end to end through the C ABI with host buffers (pinned).  Every step
-    # uploads its inputs from pinned host memory and downloads its results;
-    # as a training loop would, the copies of neighbouring steps run on a copy
-    # stream while the current step computes (inputs and outputs double-
-    # buffered on the device), and all of them are inside the timed region.
+    # uploads its inputs from pinned host memory and downloads its results, all
+    # inside the timed region.  As a training loop would, the step runs in
+    # chunks of (batch, head) rows -- heads are independent -- so copies
+    # overlap compute: the inputs of the next chunk upload on one copy stream
+    # and the outputs of the previous chunk download on another while the
+    # current chunk computes (chunk buffers double-buffered on the device).
     e2e = None
     if not args.no_e2e:
         host_in = {n: torch.empty(grid[n].shape, dtype=grid[n].dtype, pin_memory=True)
@@ -580,64 +582,96 @@ def run_nabla(args):
             host_in[n].copy_(grid[n])
         host_out = {n: torch.empty(grid["q"].shape, dtype=torch.bfloat16, pin_memory=True)
                     for n in ("o", "dq", "dk", "dv")}
-        dev_in = [grid, {n: torch.empty_like(grid[n]) for n in host_in}]
-        dev_out = [B["out"], {n: torch.empty_like(B["out"][n]) for n in host_out}]
-        copy = torch.cuda.Stream(dev)
+        nch = max(c for c in range(1, 9) if w.BH % c == 0)  # chunks per step
+        hc = w.BH // nch                                     # (batch, head) rows per chunk
+        shape_c = nabla.shape_of(1, hc, w.T, w.H, w.W, w.D, w.P)
+        rows = lambda t, c: t.view(w.BH, w.N, w.D)[c * hc:(c + 1) * hc]
+        like = lambda t: torch.empty((hc, w.N, w.D), dtype=t.dtype, device=dev)
+        C = {"flat": {n: like(grid[n]) for n in ("q", "k", "v")},
+             "o": like(grid["q"]), "lse": torch.empty((hc, w.N), dtype=torch.float32, device=dev),
+             "dq": like(grid["q"]), "dk": like(grid["q"]), "dv": like(grid["q"]),
+             "mask": nabla.alloc_mask(shape_c, dev, cols=True),
+             "ws_mask": nabla.workspace(shape_c, nabla.OP_BUILD_MASK, dev),
+             "ws_fwd": nabla.workspace(shape_c, nabla.OP_ATTN_FWD, dev),
+             "ws_bwd": nabla.workspace(shape_c, nabla.OP_ATTN_BWD, dev)}
+        dev_in = [{n: like(grid[n]) for n in host_in} for _ in range(2)]
+        dev_out = [{n: like(grid["q"]) for n in host_out} for _ in range(2)]
+        h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
         ev = lambda: torch.cuda.Event()
         in_ready = [ev(), ev()]    # inputs of buffer b uploaded
-        in_free = [ev(), ev()]     # step using input buffer b finished reading it
+        in_free = [ev(), ev()]     # chunk using input buffer b finished reading it
         out_ready = [ev(), ev()]   # outputs of buffer b written
         out_free = [ev(), ev()]    # outputs of buffer b downloaded
 
-        def upload(b, first):
-            with torch.cuda.stream(copy):
-                if not first:
-                    copy.wait_event(in_free[b])
-                for n in host_in:
-                    dev_in[b][n].copy_(host_in[n], non_blocking=True)
-                in_ready[b].record(copy)
+        def chunk_step(src, out):
+            nabla.flatten(src["v"], w.T, w.H, w.W, w.P, out=C["flat"]["v"])
+            nabla.build_mask_grid(shape_c, prm, src["q"], src["k"], q=C["flat"]["q"],
+                                  k=C["flat"]["k"], mask=C["mask"], ws=C["ws_mask"])
+            nabla.attn_fwd(shape_c, prm, C["flat"]["q"], C["flat"]["k"], C["flat"]["v"], C["mask"],
+                           o=C["o"], lse=C["lse"], ws=C["ws_fwd"])
+            nabla.attn_bwd(shape_c, prm, C["flat"]["q"], C["flat"]["k"], C["flat"]["v"], C["o"],
+                           src["dout"], C["lse"], C["mask"], dq=C["dq"], dk=C["dk"], dv=C["dv"],
+                           ws=C["ws_bwd"])
+            for n in ("o", "dq", "dk", "dv"):
+                nabla.flatten(C[n], w.T, w.H, w.W, w.P, inverse=True, out=out[n])
 
-        def download(b):
-            with torch.cuda.stream(copy):
-                copy.wait_event(out_ready[b])
+        def upload(u, first):
+            b, c = u % 2, u % nch
+            with torch.cuda.stream(h2d_s):
+                if not first:
+                    h2d_s.wait_event(in_free[b])
+                for n in host_in:
+                    dev_in[b][n].copy_(rows(host_in[n], c), non_blocking=True)
+                in_ready[b].record(h2d_s)
+
+        def download(u):
+            b, c = u % 2, u % nch
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(out_ready[b])
                 for n in host_out:
-                    host_out[n].copy_(dev_out[b][n], non_blocking=True)
-                out_free[b].record(copy)
+                    rows(host_out[n], c).copy_(dev_out[b][n], non_blocking=True)
+                out_free[b].record(d2h_s)
 
         def run(nsteps):
+            units = nsteps * nch
             upload(0, True)
-            for s in range(nsteps):
-                b = s % 2
-                if s + 1 < nsteps:
-                    upload(1 - b, s == 0)
+            for u in range(units):
+                b = u % 2
+                if u + 1 < units:
+                    upload(u + 1, u == 0)
                 stream.wait_event(in_ready[b])
-                if s >= 2:
+                if u >= 2:
                     stream.wait_event(out_free[b])
-                step(dev_in[b], out=dev_out[b])
+                chunk_step(dev_in[b], dev_out[b])
                 in_free[b].record(stream)
                 out_ready[b].record(stream)
-                download(b)
-            done = ev()
-            done.record(copy)
-            stream.wait_event(done)
+                download(u)
+            for cs in (h2d_s, d2h_s):
+                done = ev()
+                done.record(cs)
+                stream.wait_event(done)
 
         run(max(2, args.warmup // 2))
         barrier()
         a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        copy.wait_event(a)
+        h2d_s.wait_event(a)
+        d2h_s.wait_event(a)
         run(args.steps)
         b_.record(stream)
         barrier()
         e2e_ms = max_over_ranks(a.elapsed_time(b_), world, dev) / args.steps
         h2d = sum(t.numel() * t.element_size() for t in host_in.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+        # the chunked calls must give the device-resident step's results, bit for bit
+        same = all(torch.equal(host_out[n], B["out"][n].cpu()) for n in host_out)
         e2e = {"value": whole_job_tflops(job_flop, e2e_ms), "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d * world,
-               "d2h_bytes_per_step": d2h * world,
-               "copies": "pinned host <-> device on a copy stream, overlapped with the "
-                         "neighbouring steps' compute"}
-        del dev_in, dev_out
+               "d2h_bytes_per_step": d2h * world, "outputs_match_device_step": same,
+               "copies": "pinned host <-> device in %d chunks of %d (batch, head) rows per step, "
+                         "uploads and downloads on two copy streams overlapped with the "
+                         "neighbouring chunks' compute" % (nch, hc)}
+        del dev_in, dev_out, C
 
     sweep, small_cfgs = None, None
     if rank == 0 and world == 1 and not args.no_sweep:
