@@ -22,10 +22,15 @@
 //                                                        accumulators)
 // dq_kernel: one CTA per pair of temporally adjacent QUERY blocks (128 query
 //   rows), walking the union of their mask rows, one key block per tile:
-//     S = Q . K^T,  dP = dO . V^T     (Q, dO resident in TMEM as A operands)
+//     S = Q . K^T,  dP = dO . V^T     (Q, dO resident in TMEM as A operands;
+//                                      three S buffers, one dP buffer)
 //     dS = P (dP - D)                  (bf16, written over S in TMEM)
-//     dQ += dS . K                     (TMEM accumulator)
-// All waits are bounded as in the forward.
+//     dQ += dS . K                     (TMEM accumulator; issued by a second
+//                                      warp)
+// MMAs go out four per elect.sync from converged warps, whose barrier tests
+// are warp votes: the tensor core takes an N = 64 MMA only about when it
+// starts executing it, so time the issuing warp spends elsewhere is pipe
+// idle time.  All waits are bounded as in the forward.
 #include "sm100.cuh"
 
 namespace nabla {
