@@ -46,7 +46,7 @@ NCU_DRAM = {
     # pre 317.0 + 4.0 MB, dK/dV 653.4 + 292.6 MB, dQ 649.9 + 142.5 MB at 8 heads
     ("train", "attn_bwd"): {"bytes_per_head": (317.04e6 + 3.97e6 + 653.38e6 + 292.59e6
                                                + 649.92e6 + 142.47e6) / 8,
-                            "sources_sha": "c4ee656f4caa"},
+                            "sources_sha": "aae2a86a0837"},
     # 475.7 + 140.4 MB at 8 heads
     ("train", "attn_fwd"): {"bytes_per_head": (475.69e6 + 140.43e6) / 8,
                             "sources_sha": "9ea9d3d0ece4"},
